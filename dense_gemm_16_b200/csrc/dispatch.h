@@ -1,0 +1,33 @@
+// dispatch.h -- the compiled kernel instances and the tile-config table.
+#pragma once
+
+#include <cstdint>
+
+namespace dg16 {
+
+// What a launch needs to know about one compiled kernel instance.
+struct KernelEntry {
+  const void* fn;  // __global__ function
+  int smem;        // dynamic shared memory bytes
+};
+
+enum ConfigKind : int {
+  kKindSingle = 0,  // one CTA per 128 x BN tile
+  kKindSwap = 1,    // skinny problems: C^T = B^T A^T, N fills the MMA rows
+};
+
+struct Config {
+  const char* name;
+  int kind;
+  int bn;       // MMA N (Q rows per tile)
+  int stages;   // operand ring depth
+  int group_m;  // raster band height
+};
+
+// Instances, one getter per translation unit (so they compile in parallel).
+// Each returns {nullptr, 0} for a combination that was not compiled.
+KernelEntry kernels_bn256(bool q_mn, bool bf16, bool out_f32, bool grouped);
+KernelEntry kernels_bn128(bool q_mn, bool bf16, bool out_f32, bool grouped);
+KernelEntry kernels_swap(int bn, bool bf16, bool out_f32);
+
+}  // namespace dg16

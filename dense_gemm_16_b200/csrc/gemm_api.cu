@@ -1,0 +1,506 @@
+// gemm_api.cu -- the C ABI (include/dense_gemm.h): argument checks, tensor
+// maps, config choice and launches.  All compute runs in the kernels of
+// gemm_kernel.cuh; nothing here touches matrix data.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <unordered_set>
+
+#include "../../include/dense_gemm.h"
+#include "config_table.h"
+#include "dispatch.h"
+#include "gemm_kernel.cuh"
+#include "raster.h"
+
+namespace dg16 {
+
+__device__ unsigned g_status_word;  // watchdog / argument status (first error wins)
+
+// One block waits on a barrier nothing completes; the bounded wait must give
+// up and record a time-out.
+__global__ void watchdog_selftest_kernel(unsigned* status, unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ SharedCtl ctl;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    ctl.abort = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    KParams p{};
+    p.status = status;
+    p.timeout_ns = timeout_ns;
+    wait_phase(smem_u32(&bar), 0, &ctl, p, kStatusTimeoutSelftest);
+  }
+  __syncthreads();
+}
+
+
+namespace {
+
+constexpr unsigned kEpiMask = GEMM_EPI_BIAS | GEMM_EPI_RELU | GEMM_B_COL_MAJOR;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+constexpr int kMaxDevices = 64;
+
+std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+std::atomic<int> g_forced_config{-1};
+
+struct DeviceState {
+  bool ready = false;
+  int num_sms = 0;
+  unsigned* status = nullptr;
+  std::unordered_set<const void*> attr_set;  // kernels whose smem limit is raised
+};
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+int cuda_fail(cudaError_t e) {
+  (void)cudaGetLastError();  // clear a non-sticky error so later calls are unaffected
+  (void)e;
+  return GEMM_ERR_CUDA;
+}
+
+// Device state for the current device, initialised once.
+int device_state(DeviceState** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return GEMM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& s = g_dev[dev];
+  if (!s.ready) {
+    int sms = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int major = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (major != 10) return GEMM_ERR_UNSUPPORTED;  // built for sm_100a only
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_status_word);
+    if (e != cudaSuccess) return cuda_fail(e);
+    s.num_sms = sms;
+    s.status = static_cast<unsigned*>(p);
+    s.ready = true;
+  }
+  *out = &s;
+  return GEMM_OK;
+}
+
+int ensure_smem_attr(DeviceState* s, const KernelEntry& k) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (s->attr_set.count(k.fn)) return GEMM_OK;
+  cudaError_t e =
+      cudaFuncSetAttribute(k.fn, cudaFuncAttributeMaxDynamicSharedMemorySize, k.smem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  s->attr_set.insert(k.fn);
+  return GEMM_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    else
+      (void)cudaGetLastError();
+  });
+  return g_encode;
+}
+
+// A 2- or 3-D 16-bit tensor map with 128-byte swizzle and zero fill outside
+// the tensor.  dims[0] is the contiguous dimension; strides in bytes.
+int make_map(CUtensorMap* m, const void* base, bool bf16, int rank, const uint64_t* dims,
+             const uint64_t* strides_bytes, const uint32_t* box) {
+  auto enc = encoder();
+  if (!enc) return GEMM_ERR_CUDA;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                   rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int out_bytes(int dtype) { return (dtype == GEMM_F16_OUT_F32 || dtype == GEMM_BF16_OUT_F32) ? 4 : 2; }
+bool in_bf16(int dtype) { return dtype == GEMM_BF16 || dtype == GEMM_BF16_OUT_F32; }
+
+// Checks shared by gemm() and grouped_gemm() once sizes are known.
+int check_common(int N, int K, const void* A, int64_t lda, const void* B, int64_t ldb, void* C,
+                 int64_t ldc, const void* bias, unsigned epi, int dtype) {
+  if (!C) return GEMM_ERR_INVALID_ARG;
+  if ((epi & GEMM_EPI_BIAS) && !bias) return GEMM_ERR_INVALID_ARG;
+  if (ldc < N) return GEMM_ERR_INVALID_ARG;
+  if (!aligned16(C) || (ldc * out_bytes(dtype)) % 16 != 0) return GEMM_ERR_MISALIGNED;
+  if ((epi & GEMM_EPI_BIAS) && (reinterpret_cast<uintptr_t>(bias) & 1u)) return GEMM_ERR_MISALIGNED;
+  if (K > 0) {
+    if (!A || !B) return GEMM_ERR_INVALID_ARG;
+    const bool bcol = (epi & GEMM_B_COL_MAJOR) != 0;
+    if (lda < K || ldb < (bcol ? K : N)) return GEMM_ERR_INVALID_ARG;
+    if (!aligned16(A) || !aligned16(B) || lda % 8 != 0 || ldb % 8 != 0) return GEMM_ERR_MISALIGNED;
+  }
+  return GEMM_OK;
+}
+
+int check_dtype_epi(unsigned epi, int dtype) {
+  if (dtype < GEMM_F16 || dtype > GEMM_BF16_OUT_F32) return GEMM_ERR_UNSUPPORTED;
+  if (epi & ~kEpiMask) return GEMM_ERR_UNSUPPORTED;
+  return GEMM_OK;
+}
+
+// The kernel instance for a config and problem variant.
+KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool grouped) {
+  if (c.kind == kKindSwap) {
+    if (q_mn || grouped) return {nullptr, 0};  // needs column-major B
+    return kernels_swap(c.bn, bf16, f32);
+  }
+  if (c.bn == 256) return kernels_bn256(q_mn, bf16, f32, grouped);
+  if (c.bn == 128) return kernels_bn128(q_mn, bf16, f32, grouped);
+  return {nullptr, 0};
+}
+
+int launch(const KernelEntry& k, int grid, cudaStream_t stream, const CUtensorMap& tp,
+           const CUtensorMap& tq, const KParams& kp) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = k.smem;
+  cfg.stream = stream;
+  cfg.attrs = nullptr;
+  cfg.numAttrs = 0;
+  void* args[3] = {const_cast<CUtensorMap*>(&tp), const_cast<CUtensorMap*>(&tq),
+                   const_cast<KParams*>(&kp)};
+  cudaError_t e = cudaLaunchKernelExC(&cfg, k.fn, args);
+  return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
+}
+
+int select_config(int M, int N, int K, unsigned epi, bool grouped) {
+  const int forced = g_forced_config.load();
+  if (forced >= 0) return forced;
+  return table_lookup(M, N, K, (epi & GEMM_B_COL_MAJOR) != 0, grouped);
+}
+
+template <typename InT, typename OutT>
+int launch_fill(int M, int N, void* C, int64_t ldc, const void* bias, unsigned epi,
+                cudaStream_t stream) {
+  const long long total = static_cast<long long>(M) * N;
+  const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4096));
+  fill_bias_kernel<InT, OutT><<<blocks, 256, 0, stream>>>(
+      M, N, static_cast<OutT*>(C), ldc, static_cast<const InT*>(bias), static_cast<int>(epi & 3));
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
+}
+
+int fill_dispatch(int M, int N, void* C, int64_t ldc, const void* bias, unsigned epi, int dtype,
+                  cudaStream_t stream) {
+  switch (dtype) {
+    case GEMM_F16: return launch_fill<__half, __half>(M, N, C, ldc, bias, epi, stream);
+    case GEMM_BF16:
+      return launch_fill<__nv_bfloat16, __nv_bfloat16>(M, N, C, ldc, bias, epi, stream);
+    case GEMM_F16_OUT_F32: return launch_fill<__half, float>(M, N, C, ldc, bias, epi, stream);
+    default: return launch_fill<__nv_bfloat16, float>(M, N, C, ldc, bias, epi, stream);
+  }
+}
+
+template <typename InT, typename OutT>
+int launch_fill_grouped(int G, const int32_t* rows, int total, int N, void* C, int64_t ldc,
+                        const void* bias, unsigned epi, cudaStream_t stream) {
+  fill_bias_grouped_kernel<InT, OutT><<<512, 256, 0, stream>>>(
+      G, rows, total, N, static_cast<OutT*>(C), ldc, static_cast<const InT*>(bias),
+      static_cast<int>(epi & 3));
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
+}
+
+}  // namespace
+}  // namespace dg16
+
+using namespace dg16;
+
+extern "C" {
+
+const char* gemm_version(void) { return "dense_gemm_16_b200 0.1 (sm_100a, tcgen05)"; }
+
+const char* gemm_status_string(int status) {
+  switch (status) {
+    case GEMM_OK: return "GEMM_OK";
+    case GEMM_ERR_INVALID_ARG: return "GEMM_ERR_INVALID_ARG: invalid argument";
+    case GEMM_ERR_UNSUPPORTED: return "GEMM_ERR_UNSUPPORTED: unsupported dtype, flag or config";
+    case GEMM_ERR_MISALIGNED:
+      return "GEMM_ERR_MISALIGNED: pointers must be 16-byte aligned and leading dimensions "
+             "16-byte multiples";
+    case GEMM_ERR_CUDA: return "GEMM_ERR_CUDA: a CUDA call failed (or no usable device)";
+    case GEMM_ERR_DEVICE_TIMEOUT: return "GEMM_ERR_DEVICE_TIMEOUT: a kernel's bounded wait ran out";
+    default: return "unknown gemm_status";
+  }
+}
+
+int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t ldb, void* C,
+         int64_t ldc, const void* bias, unsigned epilogue, int dtype, void* stream_) {
+  int rc = check_dtype_epi(epilogue, dtype);
+  if (rc) return rc;
+  if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return GEMM_OK;
+  rc = check_common(N, K, A, lda, B, ldb, C, ldc, bias, epilogue, dtype);
+  if (rc) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc) return rc;
+  if (K == 0) return fill_dispatch(M, N, C, ldc, bias, epilogue, dtype, stream);
+
+  const bool bcol = (epilogue & GEMM_B_COL_MAJOR) != 0;
+  const bool bf16 = in_bf16(dtype);
+  const bool f32 = out_bytes(dtype) == 4;
+  const int cid = select_config(M, N, K, epilogue, false);
+  if (cid < 0 || cid >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
+  const Config& cfg = kConfigs[cid];
+  const bool swap = cfg.kind == kKindSwap;
+  const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false);
+  if (!k.fn || (swap && !bcol)) return GEMM_ERR_UNSUPPORTED;
+  rc = ensure_smem_attr(ds, k);
+  if (rc) return rc;
+
+  CUtensorMap tp, tq;
+  const uint64_t lda_b = static_cast<uint64_t>(lda) * 2, ldb_b = static_cast<uint64_t>(ldb) * 2;
+  KParams kp = {};
+  kp.M = M;
+  kp.N = N;
+  kp.K = K;
+  kp.num_kb = (K + kBK - 1) / kBK;
+  kp.group_m = cfg.group_m;
+  kp.C = C;
+  kp.ldc = ldc;
+  kp.bias = bias;
+  kp.epi = static_cast<int>(epilogue & 3);
+  kp.status = ds->status;
+  kp.timeout_ns = g_timeout_ns.load();
+  if (!swap) {
+    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
+    rc = make_map(&tp, A, bf16, 2, dA, &lda_b, bA);
+    if (rc) return rc;
+    if (bcol) {
+      const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+      const uint32_t bB[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn)};
+      rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
+    } else {
+      const uint64_t dB[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K)};
+      const uint32_t bB[2] = {64u, static_cast<uint32_t>(kBK)};
+      rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
+    }
+    if (rc) return rc;
+    kp.num_p = (M + kBM - 1) / kBM;
+    kp.num_q = (N + cfg.bn - 1) / cfg.bn;
+  } else {
+    // P = B stored N x K, Q = A (M x K); the accumulator is C^T
+    const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+    const uint32_t bB[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
+    rc = make_map(&tp, B, bf16, 2, dB, &ldb_b, bB);
+    if (rc) return rc;
+    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn)};
+    rc = make_map(&tq, A, bf16, 2, dA, &lda_b, bA);
+    if (rc) return rc;
+    kp.num_p = (N + kBM - 1) / kBM;
+    kp.num_q = (M + cfg.bn - 1) / cfg.bn;
+  }
+  kp.num_tiles = static_cast<long long>(kp.num_p) * kp.num_q;
+  const int grid = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms));
+  return launch(k, grid, stream, tp, tq, kp);
+}
+
+int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int N, int K,
+                 const void* A, int64_t lda, const void* B, int64_t ldb, int64_t stride_b,
+                 void* C, int64_t ldc, const void* bias, unsigned epilogue, int dtype,
+                 void* stream_) {
+  int rc = check_dtype_epi(epilogue, dtype);
+  if (rc) return rc;
+  if (num_groups < 1 || num_groups > kMaxGroups || !group_rows) return GEMM_ERR_INVALID_ARG;
+  if (total_rows < 0 || N < 0 || K < 0 || stride_b < 0) return GEMM_ERR_INVALID_ARG;
+  if (total_rows == 0 || N == 0) return GEMM_OK;
+  rc = check_common(N, K, A, lda, B, ldb, C, ldc, bias, epilogue, dtype);
+  if (rc) return rc;
+  if ((reinterpret_cast<uintptr_t>(group_rows) & 3u) != 0) return GEMM_ERR_MISALIGNED;
+  const bool bcol = (epilogue & GEMM_B_COL_MAJOR) != 0;
+  if (K > 0) {
+    // each group's B must fit before the next one starts
+    const int64_t one = bcol ? static_cast<int64_t>(N) * ldb : static_cast<int64_t>(K) * ldb;
+    if (num_groups > 1 && stride_b < one) return GEMM_ERR_INVALID_ARG;
+    if ((stride_b * 2) % 16 != 0) return GEMM_ERR_MISALIGNED;
+  }
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc) return rc;
+  const bool bf16 = in_bf16(dtype);
+  const bool f32 = out_bytes(dtype) == 4;
+  if (K == 0) {
+    switch (dtype) {
+      case GEMM_F16:
+        return launch_fill_grouped<__half, __half>(num_groups, group_rows, total_rows, N, C, ldc,
+                                                   bias, epilogue, stream);
+      case GEMM_BF16:
+        return launch_fill_grouped<__nv_bfloat16, __nv_bfloat16>(
+            num_groups, group_rows, total_rows, N, C, ldc, bias, epilogue, stream);
+      case GEMM_F16_OUT_F32:
+        return launch_fill_grouped<__half, float>(num_groups, group_rows, total_rows, N, C, ldc,
+                                                  bias, epilogue, stream);
+      default:
+        return launch_fill_grouped<__nv_bfloat16, float>(num_groups, group_rows, total_rows, N,
+                                                         C, ldc, bias, epilogue, stream);
+    }
+  }
+  const int cid = select_config(total_rows, N, K, epilogue, true);
+  if (cid < 0 || cid >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
+  const Config& cfg = kConfigs[cid];
+  const KernelEntry k = kernel_for(cfg, !bcol, bf16, f32, true);
+  if (!k.fn) return GEMM_ERR_UNSUPPORTED;
+  rc = ensure_smem_attr(ds, k);
+  if (rc) return rc;
+
+  CUtensorMap tp, tq;
+  const uint64_t lda_b = static_cast<uint64_t>(lda) * 2;
+  const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(total_rows)};
+  const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
+  rc = make_map(&tp, A, bf16, 2, dA, &lda_b, bA);
+  if (rc) return rc;
+  const uint64_t sB[2] = {static_cast<uint64_t>(ldb) * 2, static_cast<uint64_t>(stride_b) * 2};
+  // a single group may pass stride_b = 0; give the map a valid stride
+  uint64_t sB_fix[2] = {sB[0], num_groups > 1 ? sB[1] : (bcol ? N : K) * sB[0]};
+  if (bcol) {
+    const uint64_t dB[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                            static_cast<uint64_t>(num_groups)};
+    const uint32_t bB[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn), 1u};
+    rc = make_map(&tq, B, bf16, 3, dB, sB_fix, bB);
+  } else {
+    const uint64_t dB[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K),
+                            static_cast<uint64_t>(num_groups)};
+    const uint32_t bB[3] = {64u, static_cast<uint32_t>(kBK), 1u};
+    rc = make_map(&tq, B, bf16, 3, dB, sB_fix, bB);
+  }
+  if (rc) return rc;
+
+  KParams kp = {};
+  kp.M = total_rows;
+  kp.N = N;
+  kp.K = K;
+  kp.num_kb = (K + kBK - 1) / kBK;
+  kp.group_m = cfg.group_m;
+  kp.C = C;
+  kp.ldc = ldc;
+  kp.bias = bias;
+  kp.epi = static_cast<int>(epilogue & 3);
+  kp.group_rows = group_rows;
+  kp.num_groups = num_groups;
+  kp.status = ds->status;
+  kp.timeout_ns = g_timeout_ns.load();
+  // upper bound on tiles: each group adds at most one partial row block
+  const long long nq = (N + cfg.bn - 1) / cfg.bn;
+  const long long max_tiles = (static_cast<long long>(total_rows) / kBM + num_groups) * nq;
+  const int grid = static_cast<int>(std::min<long long>(max_tiles, ds->num_sms));
+  return launch(k, grid, stream, tp, tq, kp);
+}
+
+int gemm_device_status(void* stream_, int clear) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  unsigned w = 0;
+  e = cudaMemcpy(&w, ds->status, sizeof(w), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (clear) {
+    const unsigned zero = 0;
+    e = cudaMemcpy(ds->status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  if (w == kStatusOk) return GEMM_OK;
+  if (w == kStatusBadGroups) return GEMM_ERR_INVALID_ARG;
+  return GEMM_ERR_DEVICE_TIMEOUT;
+}
+
+uint64_t gemm_set_timeout_ns(uint64_t ns) {
+  return g_timeout_ns.exchange(ns ? ns : kDefaultTimeoutNs);
+}
+
+int gemm_watchdog_selftest(uint64_t timeout_ns, void* stream_) {
+  DeviceState* ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc) return rc;
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return GEMM_ERR_INVALID_ARG;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  watchdog_selftest_kernel<<<1, 32, 0, stream>>>(ds->status, timeout_ns);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return gemm_device_status(stream_, 1);
+}
+
+int gemm_num_configs(void) { return kNumConfigs; }
+
+int gemm_config_name(int id, char* buf, int buflen) {
+  if (id < 0 || id >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
+  if (!buf || buflen <= 0) return GEMM_ERR_INVALID_ARG;
+  std::snprintf(buf, static_cast<size_t>(buflen), "%s", kConfigs[id].name);
+  return GEMM_OK;
+}
+
+int gemm_select_config(int M, int N, int K, int dtype, unsigned epilogue) {
+  int rc = check_dtype_epi(epilogue, dtype);
+  if (rc) return rc;
+  if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
+  return select_config(M, N, K, epilogue, false);
+}
+
+int gemm_force_config(int id) {
+  if (id < -1 || id >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
+  g_forced_config.store(id);
+  return GEMM_OK;
+}
+
+int64_t gemm_smem_ring_bytes(int bm, int bn, int bk, int stages, int elem_bytes) {
+  if (bm < 0 || bn < 0 || bk < 0 || stages < 0 || elem_bytes < 0) return -1;
+  return (static_cast<int64_t>(bm) * bk + static_cast<int64_t>(bk) * bn) * elem_bytes * stages;
+}
+
+int gemm_k_iterations(int K, int bk) {
+  if (K < 0 || bk <= 0) return -1;
+  return (K + bk - 1) / bk;
+}
+
+int gemm_tile_coord(int64_t tile, int grid_m, int grid_n, int group_m, int* m_block,
+                    int* n_block) {
+  if (tile < 0 || grid_m <= 0 || grid_n <= 0 || group_m <= 0 || !m_block || !n_block)
+    return GEMM_ERR_INVALID_ARG;
+  if (tile >= static_cast<int64_t>(grid_m) * grid_n) return GEMM_ERR_INVALID_ARG;
+  int m = 0, n = 0;
+  raster_tile(tile, grid_m, grid_n, group_m, m, n);
+  *m_block = m;
+  *n_block = n;
+  return GEMM_OK;
+}
+
+}  // extern "C"

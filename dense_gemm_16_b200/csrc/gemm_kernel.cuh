@@ -1,0 +1,526 @@
+// gemm_kernel.cuh -- the persistent, warp-specialised tcgen05 GEMM kernel.
+//
+// One CTA per SM loops over output tiles.  Its six warps split the work:
+//   warp 0      TMA producer: streams 64-deep K slices of the two operands
+//               into a STAGES-deep shared-memory ring (the counterpart of the
+//               pages' num_stages software pipelining, "FlagOS众智跨芯算子优化
+//               实践" section 2.2), 128-byte swizzled so the tensor core reads
+//               them without bank conflicts (the pages' padding / XOR swizzle
+//               of section 2.3, done here by the copy engine itself).
+//   warp 1      allocates tensor memory, then one lane issues tcgen05.mma
+//               (128 x BN x 16 per instruction) into an fp32 accumulator in
+//               TMEM; two accumulators alternate so the epilogue of one tile
+//               overlaps the main loop of the next.
+//   warps 2..5  epilogue: tcgen05.ld the accumulator, add bias, ReLU, round
+//               to the output type and store ("用Triton跨芯片优化GEMM" section
+//               3.4: bias + ReLU fused after the GEMM, one trip to memory).
+// Tiles are visited in grouped-M order ("Triton 学习笔记" 2.3.7) so that the
+// tiles in flight on all SMs share operand panels in L2.
+//
+// Operand naming: the MMA computes D[p, q] = sum_k P[p, k] * Q[q, k] with P
+// the 128-row operand and Q the BN-row operand.  For C = A.B, P = A (K-major)
+// and Q = B (K-major when B is column-major, MN-major when row-major).  In
+// the swapped ("skinny") form, P = B stored N x K and Q = A, so D = C^T and the
+// wide N dimension fills the 128 MMA rows while the few rows of A become the
+// MMA's N.
+//
+// Every wait is bounded (see wait_phase); on a time-out the block records an
+// error in the device status word, drains its own asynchronous work, frees
+// its tensor memory and returns.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <type_traits>
+
+#include "ptx.cuh"
+#include "raster.h"
+
+namespace dg16 {
+
+constexpr int kBM = 128;         // MMA rows per CTA
+constexpr int kBK = 64;          // K elements per stage = one 128-byte swizzle row
+constexpr int kThreads = 192;    // 6 warps
+constexpr int kMaxGroups = 1024; // grouped GEMM: groups per launch
+
+// Device status word codes (first error wins).
+enum : unsigned {
+  kStatusOk = 0,
+  kStatusTimeoutProducer = 1,
+  kStatusTimeoutMma = 2,
+  kStatusTimeoutEpilogue = 3,
+  kStatusTimeoutSelftest = 4,
+  kStatusBadGroups = 16,
+};
+
+struct KParams {
+  int M, N, K;            // dense: problem size; grouped: total rows, N, K
+  int num_p, num_q;       // dense tile grid (P blocks x Q blocks)
+  int num_kb;             // K blocks of kBK
+  int group_m;            // raster group height
+  long long num_tiles;    // dense tile count
+  void* C;
+  long long ldc;
+  const void* bias;
+  int epi;                // bit0 bias, bit1 relu
+  const int* group_rows;  // grouped: device counts
+  int num_groups;
+  unsigned* status;       // device status word
+  unsigned long long timeout_ns;
+};
+
+struct SharedCtl {
+  int abort;
+  unsigned tmem_base;
+};
+
+// Bounded wait on an mbarrier phase.  Returns false when the block is
+// aborting (another warp gave up) or when this wait itself ran out, in which
+// case it records `code` and raises the block's abort flag.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, SharedCtl* ctl,
+                                           const KParams& p, unsigned code) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t n = 1;; ++n) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((n & 63u) == 0) {
+      if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
+      if (global_timer_ns() - t0 > p.timeout_ns) {
+        atomicCAS(p.status, 0u, code);
+        *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag: used only to drain a block's
+// own asynchronous work on the way out.
+__device__ __forceinline__ bool wait_phase_drain(uint32_t bar, uint32_t parity,
+                                                 unsigned long long limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_timer_ns() - t0 > limit_ns) return false;
+  return true;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+
+// Pack two fp32 values into the 32-bit pair of the output type (RNE).
+template <typename OutT>
+__device__ __forceinline__ uint32_t pack2(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <typename OutT>
+__device__ __forceinline__ OutT from_f32(float v);
+template <>
+__device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+template <>
+__device__ __forceinline__ float from_f32<float>(float v) { return v; }
+
+// Where a tile lives.
+struct TileCoord {
+  int p0;        // first P row (dense: global; grouped: global row of A)
+  int q0;        // first Q row
+  int group;     // grouped: group index (0 otherwise)
+  int row_end;   // grouped: one past the group's last global row
+  bool valid;
+};
+
+// Grouped-GEMM schedule: per-group tile prefix and row starts, in shared memory.
+struct GroupTable {
+  int tile_start[kMaxGroups + 1];
+  int row_start[kMaxGroups + 1];
+};
+
+template <bool GROUPED>
+__device__ __forceinline__ TileCoord tile_coord(long long t, const KParams& p, int num_q_blocks,
+                                                const GroupTable* gt, int& gcursor) {
+  TileCoord c;
+  c.group = 0;
+  c.valid = true;
+  if constexpr (!GROUPED) {
+    int pb, qb;
+    raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
+    c.p0 = pb * kBM;
+    c.q0 = qb;  // caller scales by BN
+    c.row_end = p.M;
+  } else {
+    // tiles are visited in increasing order by each role, so walk forward
+    while (gcursor < p.num_groups && t >= gt->tile_start[gcursor + 1]) ++gcursor;
+    if (gcursor >= p.num_groups) {
+      c.valid = false;
+      return c;
+    }
+    const int g = gcursor;
+    const int local = static_cast<int>(t - gt->tile_start[g]);
+    const int rows = gt->row_start[g + 1] - gt->row_start[g];
+    const int mblocks = (rows + kBM - 1) / kBM;
+    int mb, nb;
+    raster_tile(local, mblocks, num_q_blocks, p.group_m, mb, nb);
+    c.group = g;
+    c.p0 = gt->row_start[g] + mb * kBM;
+    c.q0 = nb;
+    c.row_end = min(gt->row_start[g + 1], p.M);
+  }
+  return c;
+}
+
+// The kernel.
+//   BN      Q rows per tile = MMA N (multiple of 16; of 64 when Q is MN-major)
+//   STAGES  depth of the operand ring
+//   Q_MN    Q operand is MN-major in memory (row-major B)
+//   IN_BF16 inputs are bf16 (else fp16); InT is the matching CUDA type
+//   OutT    output element type (__half, __nv_bfloat16 or float)
+//   SWAP    P = B (N x K), Q = A: the accumulator holds C^T
+//   GROUPED grouped GEMM (Q tensor map is 3-D: [group][rows][K or N])
+template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT, bool SWAP, bool GROUPED>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
+                   const KParams p) {
+  using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
+  static_assert(!Q_MN || BN % 64 == 0, "MN-major Q tiles are whole 64-element swizzle rows");
+  static_assert(!(SWAP && GROUPED), "grouped GEMM uses the plain operand order");
+  constexpr uint32_t P_BYTES = kBM * kBK * 2;
+  constexpr uint32_t Q_BYTES = BN * kBK * 2;
+  constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
+  constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
+                                 : (2 * BN <= 256) ? 256 : 512;
+  constexpr uint32_t IDESC = f16_idesc(kBM, BN, IN_BF16 ? 1u : 0u, 0u, Q_MN ? 1u : 0u);
+
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128-byte swizzle atoms (8 rows x 128 B)
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sP = smem;
+  uint8_t* sQ = smem + STAGES * P_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sQ + STAGES * Q_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + STAGES;
+  uint64_t* accf_bar = bars + 2 * STAGES;
+  uint64_t* acce_bar = bars + 2 * STAGES + 2;
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;
+  SharedCtl* ctl = reinterpret_cast<SharedCtl*>(bars + 2 * STAGES + 5);
+  GroupTable* gt = reinterpret_cast<GroupTable*>(ctl + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&accf_bar[a]), 1);
+      mbar_init(smem_u32(&acce_bar[a]), 4 * 32);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmP);
+    tma_prefetch_desc(&tmQ);
+  }
+  if (warp == 1) {
+    tmem_alloc<1>(smem_u32(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish<1>();
+  }
+  if constexpr (GROUPED) {
+    if (warp == 2 && lane == 0) {
+      // per-group tile prefix from the device counts (no host sync)
+      int tiles = 0, rows = 0;
+      const int nq = (p.N + BN - 1) / BN;
+      bool bad = false;
+      for (int g = 0; g < p.num_groups; ++g) {
+        int m = __ldg(&p.group_rows[g]);
+        if (m < 0) {
+          m = 0;
+          bad = true;
+        }
+        gt->tile_start[g] = tiles;
+        gt->row_start[g] = rows;
+        // rows past the stated total are never read or written
+        const int usable = max(0, min(m, p.M - rows));
+        if (usable < m) bad = true;
+        tiles += (usable + kBM - 1) / kBM * nq;
+        rows += usable;
+      }
+      gt->tile_start[p.num_groups] = tiles;
+      gt->row_start[p.num_groups] = rows;
+      if (bad && blockIdx.x == 0) atomicCAS(p.status, 0u, kStatusBadGroups);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  long long num_tiles = p.num_tiles;
+  if constexpr (GROUPED) num_tiles = gt->tile_start[p.num_groups];
+  const int num_q_blocks = GROUPED ? (p.N + BN - 1) / BN : p.num_q;
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      // A/B panels are re-read by the tiles of the same raster group: keep
+      // them in L2 ahead of the streaming output.
+      const uint64_t pol = policy_evict_last();
+      uint32_t it = 0;
+      int gcur = 0;
+      bool ok = true;
+      for (long long t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
+        if (!c.valid) break;
+        const int q0 = c.q0 * BN;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_phase(smem_u32(&empty_bar[s]), ph ^ 1u, ctl, p, kStatusTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          mbar_arrive_expect_tx(fb, STAGE_BYTES);
+          tma_load_2d(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, c.p0, fb, pol);
+          const uint32_t qdst = smem_u32(sQ + s * Q_BYTES);
+          if constexpr (GROUPED) {
+            if constexpr (Q_MN) {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j)
+                tma_load_3d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, c.group, fb,
+                            pol);
+            } else {
+              tma_load_3d(qdst, &tmQ, kb * kBK, q0, c.group, fb, pol);
+            }
+          } else {
+            if constexpr (Q_MN) {
+#pragma unroll
+              for (int j = 0; j < BN / 64; ++j)
+                tma_load_2d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, fb, pol);
+            } else {
+              tma_load_2d(qdst, &tmQ, kb * kBK, q0, fb, pol);
+            }
+          }
+        }
+      }
+      if (!ok) {
+        // leave no copy in flight into this block's shared memory
+        const uint32_t first = it > STAGES ? it - STAGES : 0;
+        for (uint32_t j = first; j < it; ++j)
+          wait_phase_drain(smem_u32(&full_bar[j % STAGES]), (j / STAGES) & 1u, 50000000ull);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, local = 0;
+      int gcur = 0;
+      bool ok = true;
+      for (long long t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+        const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
+        if (!c.valid) break;
+        const uint32_t a = local & 1u;
+        const uint32_t aph = (local >> 1) & 1u;
+        if (!wait_phase(smem_u32(&acce_bar[a]), aph ^ 1u, ctl, p, kStatusTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + a * BN;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_phase(smem_u32(&full_bar[s]), ph, ctl, p, kStatusTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pbase = smem_u32(sP + s * P_BYTES);
+          const uint32_t qbase = smem_u32(sQ + s * Q_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            // K-major: the k-th 16-element slice starts 32 bytes further
+            // along each 128-byte swizzled row; 8-row groups are 1024 B apart.
+            const uint64_t adesc = sw128_desc(pbase + k * 32, 16, 1024);
+            // MN-major: 16 K rows of 128 B per slice; 64-element MN chunks are
+            // kBK rows apart; 8-row K groups 1024 B apart.
+            const uint64_t bdesc = Q_MN ? sw128_desc(qbase + k * 16 * 128, kBK * 128, 1024)
+                                        : sw128_desc(qbase + k * 32, 16, 1024);
+            mma_f16<1>(d, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          mma_commit<1>(smem_u32(&empty_bar[s]));  // frees the stage when read
+        }
+        if (!ok) break;
+        mma_commit<1>(smem_u32(&accf_bar[a]));  // accumulator ready
+      }
+      // every MMA this thread issued has completed before tensor memory is freed
+      mma_commit<1>(smem_u32(drain_bar));
+      wait_phase_drain(smem_u32(drain_bar), 0, 50000000ull);
+    }
+    __syncwarp();
+  } else {
+    // ----------------------------------------------------------- epilogue
+    const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
+    uint32_t local = 0;
+    int gcur = 0;
+    OutT* C = reinterpret_cast<OutT*>(p.C);
+    const InT* bias = reinterpret_cast<const InT*>(p.bias);
+    const bool has_bias = (p.epi & 1) != 0;
+    const bool relu = (p.epi & 2) != 0;
+    for (long long t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+      const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
+      if (!c.valid) break;
+      const uint32_t a = local & 1u;
+      const uint32_t aph = (local >> 1) & 1u;
+      // every lane waits; the warp proceeds only if all saw the phase, so the
+      // .sync.aligned TMEM loads below are always issued by the whole warp
+      const bool ok = wait_phase(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int prow = c.p0 + quad * 32 + lane;  // this thread's accumulator row
+      const int q0 = c.q0 * BN;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * BN;
+      if constexpr (!SWAP) {
+        // accumulator row = output row prow, columns q0 .. q0+BN
+        const bool row_ok = prow < c.row_end;
+        const InT* bias_g = has_bias ? bias + static_cast<long long>(c.group) * p.N : nullptr;
+        OutT* crow = C + static_cast<long long>(prow) * p.ldc;
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 32) {
+          const int col0 = q0 + cc;
+          if (col0 >= p.N) break;  // warp-uniform
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(taddr + cc, v);
+          tmem_ld_wait();
+          float f[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            float x = __uint_as_float(v[j]);
+            if (has_bias && col0 + j < p.N) x += to_f32<InT>(bias_g[col0 + j]);
+            if (relu) x = fmaxf(x, 0.0f);
+            f[j] = x;
+          }
+          if (row_ok) {
+            if (col0 + 32 <= p.N) {
+              if constexpr (sizeof(OutT) == 2) {
+                uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                  dst[j] = make_uint4(pack2<OutT>(f[8 * j + 0], f[8 * j + 1]),
+                                      pack2<OutT>(f[8 * j + 2], f[8 * j + 3]),
+                                      pack2<OutT>(f[8 * j + 4], f[8 * j + 5]),
+                                      pack2<OutT>(f[8 * j + 6], f[8 * j + 7]));
+              } else {
+                float4* dst = reinterpret_cast<float4*>(crow + col0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                  dst[j] = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j < p.N) crow[col0 + j] = from_f32<OutT>(f[j]);
+            }
+          }
+        }
+      } else {
+        // accumulator row = output column prow (an N index); accumulator
+        // columns are output rows q0 .. q0+BN
+        const bool col_ok = prow < p.N;
+        const float b = (has_bias && col_ok) ? to_f32<InT>(bias[prow]) : 0.0f;
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 16) {
+          const int row0 = q0 + cc;
+          if (row0 >= p.M) break;  // warp-uniform
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(taddr + cc, v);
+          tmem_ld_wait();
+          if (col_ok) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (row0 + j < p.M) {
+                float x = __uint_as_float(v[j]) + b;
+                if (relu) x = fmaxf(x, 0.0f);
+                C[static_cast<long long>(row0 + j) * p.ldc + prow] = from_f32<OutT>(x);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&acce_bar[a]));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc<1>(tmem_base, TMEM_COLS);
+  }
+}
+
+// Shared memory a kernel instance needs (bytes, including alignment slack).
+template <int BN, int STAGES, bool GROUPED>
+constexpr int gemm_smem_bytes() {
+  return 1024 + STAGES * (kBM * kBK * 2 + BN * kBK * 2) + (2 * STAGES + 5) * 8 +
+         static_cast<int>(sizeof(SharedCtl)) + (GROUPED ? static_cast<int>(sizeof(GroupTable)) : 0);
+}
+
+// C = act(bias) (or zeros) for K == 0: the definition with an empty sum.
+template <typename InT, typename OutT>
+__global__ void fill_bias_kernel(int M, int N, OutT* C, long long ldc, const InT* bias, int epi) {
+  const long long total = static_cast<long long>(M) * N;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int r = static_cast<int>(i / N), c = static_cast<int>(i % N);
+    float x = (epi & 1) ? to_f32<InT>(bias[c]) : 0.0f;
+    if (epi & 2) x = fmaxf(x, 0.0f);
+    C[static_cast<long long>(r) * ldc + c] = from_f32<OutT>(x);
+  }
+}
+
+// Grouped K == 0: every stored row gets act(bias_g).
+template <typename InT, typename OutT>
+__global__ void fill_bias_grouped_kernel(int num_groups, const int* group_rows, int total_rows,
+                                         int N, OutT* C, long long ldc, const InT* bias, int epi) {
+  int row0 = 0;
+  for (int g = 0; g < num_groups; ++g) {
+    const int m = max(0, min(group_rows[g], total_rows - row0));
+    const long long total = static_cast<long long>(m) * N;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<long long>(gridDim.x) * blockDim.x) {
+      const int r = row0 + static_cast<int>(i / N), c = static_cast<int>(i % N);
+      float x = (epi & 1) ? to_f32<InT>(bias[static_cast<long long>(g) * N + c]) : 0.0f;
+      if (epi & 2) x = fmaxf(x, 0.0f);
+      C[static_cast<long long>(r) * ldc + c] = from_f32<OutT>(x);
+    }
+    row0 += m;
+  }
+}
+
+}  // namespace dg16

@@ -1,0 +1,216 @@
+/*
+ * dense_gemm.h -- C ABI of the B200 (sm_100a) tiled GEMM library.
+ *
+ * The operation is the tiled dense GEMM the pages build in Triton:
+ *
+ *     C = act(A . B + bias)          act = identity or ReLU
+ *
+ * with fp16 or bf16 inputs and an fp32 accumulator ("用Triton跨芯片优化GEMM：
+ * 实测性能反超原生算子库", section 2.1 for the tiled product with an fp32
+ * accumulator and section 3.4 for the bias + ReLU epilogue fused into the
+ * same kernel; "Triton 学习笔记", section 2.1: always accumulate in fp32).
+ * The grouped entry point runs the many GEMMs of an MoE layer in a single
+ * launch (first page, section 2.3).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout.   All matrices are addressed through a leading dimension, in
+ *           elements, the way the pages pass a stride per dimension
+ *           ("Triton 学习笔记" section 1, strides and transposes):
+ *             A[i,k] = A[i*lda + k]                        (row-major, M x K)
+ *             B[k,j] = B[k*ldb + j]                        (row-major, K x N)
+ *             B[k,j] = B[j*ldb + k]  with GEMM_B_COL_MAJOR (stored N x K)
+ *             C[i,j] = C[i*ldc + j]                        (row-major, M x N)
+ *           bias is a length-N vector of the input type, broadcast over rows.
+ * Memory.   Every pointer except the grouped call's host scalars is a DEVICE
+ *           pointer owned by the caller.  The library never allocates,
+ *           frees or keeps a reference to a caller buffer after the call.
+ * Alignment. A, B and C must be 16-byte aligned; lda and ldb must be
+ *           multiples of 8 elements and ldc*sizeof(output) a multiple of 16
+ *           bytes (the tensor-memory-access unit copies 16-byte granules).
+ *           bias needs only its element alignment.  Anything else returns
+ *           GEMM_ERR_MISALIGNED; there is no slower fallback.
+ * Sizes.    M, N, K >= 0.  M == 0 or N == 0 is a no-op that returns GEMM_OK.
+ *           K == 0 writes C = act(bias) (or 0) -- the plain definition.
+ * Streams.  `stream` is a cudaStream_t (NULL = the legacy default stream).
+ *           Calls are asynchronous: GEMM_OK means the work was enqueued;
+ *           a device-side fault shows up at the caller's next synchronisation,
+ *           and a watchdog time-out is reported by gemm_device_status().
+ * Errors.   Every function returns a gemm_status; nothing throws, aborts or
+ *           exits.  Argument errors are detected before anything is launched.
+ * Threads.  All entry points are thread-safe.  The only mutable global state
+ *           is a per-device cache (SM count, status-word address, kernel
+ *           attributes) filled once per device, and the config override.
+ */
+#ifndef DENSE_GEMM_H
+#define DENSE_GEMM_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define GEMM_API __attribute__((visibility("default")))
+#else
+#define GEMM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  GEMM_OK = 0,
+  GEMM_ERR_INVALID_ARG = -1,    /* null pointer, negative size, ld too small */
+  GEMM_ERR_UNSUPPORTED = -2,    /* unknown dtype, epilogue bit or config id */
+  GEMM_ERR_MISALIGNED = -3,     /* pointer or leading dimension breaks the 16-byte rule */
+  GEMM_ERR_CUDA = -4,           /* a CUDA runtime / driver call failed (incl. no device) */
+  GEMM_ERR_DEVICE_TIMEOUT = -5  /* a kernel's bounded wait ran out (see gemm_device_status) */
+} gemm_status;
+
+typedef enum {
+  GEMM_F16 = 0,          /* fp16 in, fp32 accumulate, fp16 out (round to nearest even) */
+  GEMM_BF16 = 1,         /* bf16 in, fp32 accumulate, bf16 out (round to nearest even) */
+  GEMM_F16_OUT_F32 = 2,  /* fp16 in, fp32 accumulate, fp32 out */
+  GEMM_BF16_OUT_F32 = 3  /* bf16 in, fp32 accumulate, fp32 out */
+} gemm_dtype;
+
+/* `epilogue` bits. */
+#define GEMM_EPI_BIAS 0x1u     /* add bias[j] (input dtype) to every row, in fp32 */
+#define GEMM_EPI_RELU 0x2u     /* then max(x, 0), before the output cast */
+#define GEMM_B_COL_MAJOR 0x100u /* B is stored N x K: B[k,j] = B[j*ldb + k] */
+
+/*
+ * gemm -- C = act(A . B + bias) on one GPU, one launch.
+ *
+ * Defined by "用Triton跨芯片优化GEMM" section 2.1 (tiled GEMM, fp32
+ * accumulator) and section 3.4 (bias and ReLU applied to the accumulator
+ * inside the kernel before the single store).  The result of each element is
+ * the exact sum of its K products rounded only by the fp32 accumulation (in
+ * an unspecified order) and by the final cast.
+ *
+ *   M, N, K   problem size (elements), each >= 0
+ *   A         device, M x K, leading dimension lda (>= K when K > 0)
+ *   B         device, K x N row-major with ldb >= N, or N x K (ldb >= K)
+ *             with GEMM_B_COL_MAJOR
+ *   C         device, M x N, ldc >= N, output dtype per `dtype`; C must not
+ *             overlap A, B or bias
+ *   bias      device, N elements of the input dtype; required iff
+ *             GEMM_EPI_BIAS, ignored otherwise
+ *   epilogue  OR of GEMM_EPI_BIAS, GEMM_EPI_RELU, GEMM_B_COL_MAJOR
+ *   dtype     a gemm_dtype
+ *   stream    cudaStream_t
+ * Returns GEMM_OK or an error status; on error nothing was launched.
+ */
+GEMM_API int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t ldb, void* C,
+         int64_t ldc, const void* bias, unsigned epilogue, int dtype, void* stream);
+
+/*
+ * grouped_gemm -- the per-expert GEMMs of an MoE layer in one launch
+ * ("用Triton跨芯片优化GEMM" section 2.3: a MoE layer runs dozens of GEMMs).
+ *
+ * Rows of A (and C) are sorted by group: group g owns rows
+ * [r_g, r_g + group_rows[g]) with r_g = sum_{h<g} group_rows[h], and
+ *     C[r, :] = act(A[r, :] . B_g + bias_g)   for every row r of group g,
+ * B_g = B + g*stride_b (same layout rules as gemm(), ldb shared by all
+ * groups), bias_g = bias + g*N.
+ *
+ *   num_groups  1..1024
+ *   group_rows  DEVICE int32[num_groups]; read by the kernel, so a routing
+ *               step earlier on the same stream may produce it (no host sync)
+ *   total_rows  host int, the rows of A and C (= sum of group_rows); rows the
+ *               device counts place beyond total_rows are neither read nor
+ *               written, and a negative count is treated as 0 -- both set
+ *               the device status (gemm_device_status) to GEMM_ERR_INVALID_ARG
+ *   N, K        per-group GEMM size (shared by all groups)
+ *   A, lda      device, total_rows x K
+ *   B, ldb      device, num_groups matrices, each K x N (or N x K with
+ *               GEMM_B_COL_MAJOR); stride_b elements apart (stride_b*2 a
+ *               multiple of 16 bytes)
+ *   C, ldc      device, total_rows x N
+ *   bias        device, num_groups x N (input dtype) iff GEMM_EPI_BIAS
+ * Empty groups cost nothing; rows of a group's last tile that belong to the
+ * next group are computed but never stored.
+ */
+GEMM_API int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int N, int K,
+                 const void* A, int64_t lda, const void* B, int64_t ldb, int64_t stride_b,
+                 void* C, int64_t ldc, const void* bias, unsigned epilogue, int dtype,
+                 void* stream);
+
+/* Human-readable name of a gemm_status value (static storage). */
+GEMM_API const char* gemm_status_string(int status);
+
+/* Library version string (static storage). */
+GEMM_API const char* gemm_version(void);
+
+/*
+ * gemm_device_status -- synchronise `stream`, then read the current device's
+ * status word that the kernels' watchdogs and argument checks write.  Returns
+ * GEMM_OK, GEMM_ERR_DEVICE_TIMEOUT (a bounded wait inside a kernel ran out
+ * and the kernel returned early; its output is undefined) or
+ * GEMM_ERR_INVALID_ARG (grouped row counts were inconsistent).  With clear
+ * != 0 the word is reset to 0 afterwards.
+ */
+GEMM_API int gemm_device_status(void* stream, int clear);
+
+/*
+ * gemm_set_timeout_ns -- bound, in nanoseconds, of every wait inside the
+ * kernels (default 2e9).  A wait that runs out sets the device status word,
+ * and every warp of that block leaves its loop, waits (again bounded) for
+ * its own copies and MMAs in flight, frees its tensor memory and returns.
+ * 0 restores the default.  Returns the previous value.
+ */
+GEMM_API uint64_t gemm_set_timeout_ns(uint64_t ns);
+
+/*
+ * gemm_watchdog_selftest -- launch one block whose wait is on a barrier that
+ * nothing ever completes, with the given bound; the kernel must give up,
+ * record GEMM_ERR_DEVICE_TIMEOUT and return.  Synchronises `stream` and
+ * returns what gemm_device_status(stream, 1) then reports (expected:
+ * GEMM_ERR_DEVICE_TIMEOUT).  No fault, trap or hang is involved.
+ */
+GEMM_API int gemm_watchdog_selftest(uint64_t timeout_ns, void* stream);
+
+/* ---- tile configurations (the offline sweep's table) ------------------- */
+
+/* Number of tile configurations compiled into the library. */
+GEMM_API int gemm_num_configs(void);
+
+/* Name of configuration `id` into buf (NUL-terminated, truncated to
+ * buflen); returns GEMM_OK or GEMM_ERR_UNSUPPORTED for a bad id. */
+GEMM_API int gemm_config_name(int id, char* buf, int buflen);
+
+/* Id of the configuration gemm() would use for this problem (the table's
+ * choice, or the forced id), or a negative gemm_status if none applies. */
+GEMM_API int gemm_select_config(int M, int N, int K, int dtype, unsigned epilogue);
+
+/* Force every later gemm() / grouped_gemm() call in this process onto
+ * configuration `id` (-1 restores the table).  For the offline sweep and for
+ * tests; a forced config that cannot run a problem makes that call return
+ * GEMM_ERR_UNSUPPORTED.  Returns GEMM_OK or GEMM_ERR_UNSUPPORTED. */
+GEMM_API int gemm_force_config(int id);
+
+/* ---- host-side helpers (no GPU needed) --------------------------------- */
+
+/* Bytes of the shared-memory operand ring for a BM x BN output tile with a
+ * BK-deep K step and `stages` buffers: (BM*BK + BK*BN) * elem_bytes * stages,
+ * the formula of the crowd-sourced tuning page ("FlagOS众智跨芯算子优化实践",
+ * section 2.1; its worked example 128/128/32, fp16, 3 stages = 49152 bytes).
+ * Returns -1 on a negative argument. */
+GEMM_API int64_t gemm_smem_ring_bytes(int bm, int bn, int bk, int stages, int elem_bytes);
+
+/* K-loop trip count ceil(K / bk) (same page, section 2.2: K = 512 with
+ * BLOCK_K = 64 runs 8 iterations).  Returns -1 on a bad argument. */
+GEMM_API int gemm_k_iterations(int K, int bk);
+
+/* Grouped-M rasterisation of a linear tile index onto a grid_m x grid_n tile
+ * grid, groups of group_m tile rows walked column by column ("Triton 学习笔记"
+ * section 2.3.7 on L2 reuse; the grouped pid mapping of the Gluon/Triton
+ * page's matmul example).  Writes the tile's row and column block.  Returns
+ * GEMM_OK or GEMM_ERR_INVALID_ARG. */
+GEMM_API int gemm_tile_coord(int64_t tile, int grid_m, int grid_n, int group_m, int* m_block,
+                    int* n_block);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DENSE_GEMM_H */

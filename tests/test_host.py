@@ -1,0 +1,168 @@
+"""Host-side checks of the C-ABI library (no GPU needed): it loads, exports
+every function include/dense_gemm.h declares, its host helpers reproduce the
+pages' worked numbers, and every argument error is reported before anything
+touches CUDA."""
+import ctypes
+import os
+
+import pytest
+
+import dense_gemm_16_b200 as dg
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built_library():
+    if not os.path.exists(dg.LIB_PATH):
+        from dense_gemm_16_b200 import build
+        build.build()
+    return dg.lib()
+
+
+def test_exports_every_declared_symbol():
+    names = dg.header_functions()
+    assert {"gemm", "grouped_gemm", "gemm_status_string"} <= set(names)
+    L = dg.lib()
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+
+
+def test_version_and_status_strings():
+    assert "sm_100a" in dg.gemm_version()
+    for s in [0, -1, -2, -3, -4, -5]:
+        assert dg.gemm_status_string(s).startswith("GEMM_")
+    assert "unknown" in dg.gemm_status_string(12345)
+
+
+def _golden_rows(kind):
+    with open(os.path.join(GOLDEN, "pages_worked_numbers.txt")) as f:
+        for line in f:
+            if line.startswith(kind + " "):
+                yield dict(kv.split("=") for kv in line.split()[1:])
+
+
+def test_pages_smem_formula():
+    rows = list(_golden_rows("smem_ring"))
+    assert rows
+    for r in rows:
+        got = dg.gemm_smem_ring_bytes(int(r["BM"]), int(r["BN"]), int(r["BK"]),
+                                      int(r["stages"]), int(r["elem_bytes"]))
+        assert got == int(r["expect"])
+    assert dg.gemm_smem_ring_bytes(-1, 1, 1, 1, 1) == -1
+
+
+def test_pages_k_iterations():
+    for r in _golden_rows("k_iters"):
+        assert dg.gemm_k_iterations(int(r["K"]), int(r["BK"])) == int(r["expect"])
+    assert dg.gemm_k_iterations(2000, 64) == 32  # ragged K rounds up
+    assert dg.gemm_k_iterations(1, 0) == -1
+
+
+def test_pages_raster_block_counts():
+    """9x9 tile grid: the first 9 tiles read 90 input blocks in row-major
+    order and 54 in 3x3 grouped order (9 K-blocks per panel)."""
+    for r in _golden_rows("raster"):
+        gm, gn, tiles, kb = (int(r[k]) for k in ("grid_m", "grid_n", "tiles", "k_blocks"))
+        coords = [dg.gemm_tile_coord(t, gm, gn, int(r["group_m"])) for t in range(tiles)]
+        a_panels = {m for m, _ in coords}
+        b_panels = {n for _, n in coords}
+        assert (len(a_panels) + len(b_panels)) * kb == int(r["expect"])
+
+
+@pytest.mark.parametrize("gm,gn,group", [(9, 9, 3), (7, 5, 8), (32, 16, 8), (5, 1, 4), (1, 7, 1)])
+def test_raster_is_a_permutation(gm, gn, group):
+    seen = {dg.gemm_tile_coord(t, gm, gn, group) for t in range(gm * gn)}
+    assert seen == {(m, n) for m in range(gm) for n in range(gn)}
+
+
+def test_raster_group_one_is_row_major():
+    for t in range(35):
+        assert dg.gemm_tile_coord(t, 5, 7, 1) == (t // 7, t % 7)
+
+
+def test_configs_listed_and_forcing_bounds():
+    n = dg.gemm_num_configs()
+    assert n >= 3
+    names = [dg.gemm_config_name(i) for i in range(n)]
+    assert len(set(names)) == n
+    with pytest.raises(dg.GemmError):
+        dg.gemm_config_name(n)
+    assert dg.gemm_force_config(n) == dg.GEMM_ERR_UNSUPPORTED
+    assert dg.gemm_force_config(-2) == dg.GEMM_ERR_UNSUPPORTED
+    assert dg.gemm_force_config(0) == 0
+    assert dg.gemm_select_config(4096, 4096, 4096, dg.GEMM_BF16, 0) == 0
+    assert dg.gemm_force_config(-1) == 0
+
+
+def test_select_config_shape_classes():
+    bcol = dg.GEMM_B_COL_MAJOR
+    skinny = dg.gemm_select_config(16, 8192, 8192, dg.GEMM_F16, bcol)
+    assert dg.gemm_config_name(skinny).startswith("swap")
+    big = dg.gemm_select_config(8192, 8192, 8192, dg.GEMM_BF16, 0)
+    assert not dg.gemm_config_name(big).startswith("swap")
+    assert dg.gemm_select_config(-1, 1, 1, 0, 0) == dg.GEMM_ERR_INVALID_ARG
+    assert dg.gemm_select_config(1, 1, 1, 9, 0) == dg.GEMM_ERR_UNSUPPORTED
+
+
+# Fake, never-dereferenced device addresses: every case below must be
+# rejected by the host checks before any CUDA call.
+P = 1 << 20  # 16-byte aligned
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (M, N, K, A, lda, B, ldb, C, ldc, bias, epi, dtype)
+    ((4, 4, 4, P, 8, P, 8, P, 8, None, 0, 7), dg.GEMM_ERR_UNSUPPORTED),           # dtype
+    ((4, 4, 4, P, 8, P, 8, P, 8, None, 0x10, 0), dg.GEMM_ERR_UNSUPPORTED),        # epilogue bit
+    ((-1, 4, 4, P, 8, P, 8, P, 8, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),          # negative M
+    ((4, 4, -3, P, 8, P, 8, P, 8, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),          # negative K
+    ((4, 4, 4, None, 8, P, 8, P, 8, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),        # null A
+    ((4, 4, 4, P, 8, None, 8, P, 8, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),        # null B
+    ((4, 4, 4, P, 8, P, 8, None, 8, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),        # null C
+    ((4, 4, 4, P, 8, P, 8, P, 8, None, 1, 0), dg.GEMM_ERR_INVALID_ARG),           # bias flag, no bias
+    ((4, 4, 16, P, 8, P, 8, P, 8, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),          # lda < K
+    ((4, 16, 4, P, 8, P, 8, P, 16, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),         # ldb < N
+    ((4, 4, 16, P, 16, P, 8, P, 8, None, 0x100, 0), dg.GEMM_ERR_INVALID_ARG),     # col-major ldb < K
+    ((4, 16, 4, P, 8, P, 16, P, 8, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),         # ldc < N
+    ((4, 4, 4, P + 2, 8, P, 8, P, 8, None, 0, 0), dg.GEMM_ERR_MISALIGNED),        # A pointer
+    ((4, 4, 4, P, 8, P + 8, 8, P, 8, None, 0, 0), dg.GEMM_ERR_MISALIGNED),        # B pointer
+    ((4, 4, 4, P, 8, P, 8, P + 4, 8, None, 0, 0), dg.GEMM_ERR_MISALIGNED),        # C pointer
+    ((4, 4, 4, P, 12, P, 8, P, 8, None, 0, 0), dg.GEMM_ERR_MISALIGNED),           # lda % 8
+    ((4, 4, 4, P, 8, P, 10, P, 8, None, 0, 0), dg.GEMM_ERR_MISALIGNED),           # ldb % 8
+    ((4, 4, 4, P, 8, P, 8, P, 6, None, 0, 0), dg.GEMM_ERR_MISALIGNED),            # ldc*2 % 16
+    ((4, 4, 4, P, 8, P, 8, P, 6, None, 0, 2), dg.GEMM_ERR_MISALIGNED),            # ldc*4 % 16 (f32)
+    ((4, 4, 4, P, 8, P, 8, P, 8, P + 1, 1, 0), dg.GEMM_ERR_MISALIGNED),           # bias alignment
+])
+def test_gemm_argument_errors(args, expect):
+    M, N, K, A, lda, B, ldb, C, ldc, bias, epi, dtype = args
+    assert dg.lib().gemm(M, N, K, A, lda, B, ldb, C, ldc, bias, epi, dtype, None) == expect
+
+
+def test_gemm_empty_is_a_noop_without_touching_cuda():
+    L = dg.lib()
+    assert L.gemm(0, 5, 5, None, 0, None, 0, None, 0, None, 0, 0, None) == 0
+    assert L.gemm(5, 0, 5, None, 0, None, 0, None, 0, None, 0, 0, None) == 0
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (G, rows, total, N, K, A, lda, B, ldb, stride_b, C, ldc, bias, epi, dtype)
+    ((0, P, 8, 8, 8, P, 8, P, 8, 64, P, 8, None, 0, 1), dg.GEMM_ERR_INVALID_ARG),      # no groups
+    ((1025, P, 8, 8, 8, P, 8, P, 8, 64, P, 8, None, 0, 1), dg.GEMM_ERR_INVALID_ARG),   # too many
+    ((2, None, 8, 8, 8, P, 8, P, 8, 64, P, 8, None, 0, 1), dg.GEMM_ERR_INVALID_ARG),   # null rows
+    ((2, P, -1, 8, 8, P, 8, P, 8, 64, P, 8, None, 0, 1), dg.GEMM_ERR_INVALID_ARG),     # total < 0
+    ((2, P, 8, 8, 8, P, 8, P, 8, 56, P, 8, None, 0, 1), dg.GEMM_ERR_INVALID_ARG),      # overlapping B
+    ((2, P, 8, 8, 8, P, 8, P, 8, 68, P, 8, None, 0, 1), dg.GEMM_ERR_MISALIGNED),       # stride_b*2 % 16
+    ((2, P + 2, 8, 8, 8, P, 8, P, 8, 64, P, 8, None, 0, 1), dg.GEMM_ERR_MISALIGNED),   # rows pointer
+    ((2, P, 8, 8, 8, P, 8, P, 8, 64, P, 8, None, 0, 5), dg.GEMM_ERR_UNSUPPORTED),      # dtype
+])
+def test_grouped_argument_errors(args, expect):
+    assert dg.lib().grouped_gemm(*args, None) == expect
+
+
+def test_valid_call_without_a_device_reports_cuda_error():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a device is present")
+    L = dg.lib()
+    assert L.gemm(4, 4, 4, P, 8, P, 8, P, 8, None, 0, 0, None) == dg.GEMM_ERR_CUDA
+    assert L.gemm_device_status(None, 0) == dg.GEMM_ERR_CUDA

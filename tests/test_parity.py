@@ -1,0 +1,259 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, on
+the seeded workloads (every element for the small configurations, a seeded
+sample of 4096 outputs plus tile-boundary rows/columns for the large ones),
+bit-exact integer cases, edge cases, every compiled tile config, and
+sentinel guard bands around C to catch any store outside it."""
+import numpy as np
+import pytest
+import torch
+
+import dense_gemm_16_b200 as dg
+import oracle
+import workloads
+from gpu_helpers import THREADS, Guarded, compare, in_name, pad_cols, run_gemm
+
+pytestmark = pytest.mark.gpu
+
+
+def _dense_case(w, sampled: bool):
+    A, B, bias = workloads.make_inputs(w)
+    dA, dB = A.cuda(), B.cuda()
+    dbias = bias.cuda() if bias is not None else None
+    g = run_gemm(dA, dB, dbias, w.M, w.N, w.K, b_col=w.b_colmajor, relu=w.relu)
+    got = g.matrix().double().cpu().numpy()
+    g.check_canaries()
+    ldb = w.K if w.b_colmajor else w.N
+    if not sampled:
+        ref = oracle.gemm(w.M, w.N, w.K, A, w.K, B, ldb, b_colmajor=w.b_colmajor, bias=bias,
+                          relu=w.relu, dtype=w.dtype, threads=THREADS)
+        compare(got, ref, 2, w.name)
+    else:
+        rows, cols = workloads.sample_indices(w.M, w.N)
+        ref = oracle.gemm_at(w.M, w.N, w.K, A, w.K, B, ldb, rows, cols,
+                             b_colmajor=w.b_colmajor, bias=bias, relu=w.relu, dtype=w.dtype,
+                             threads=THREADS)
+        compare(got[rows, cols], ref, 2, w.name)
+    assert np.isfinite(got).all()
+
+
+@pytest.mark.parametrize("name", ["square256_f16", "m1024n1024k2048_f16",
+                                  "m1024n1024k2048_f16_bias_relu", "m1000n1000k2000_f16_bcol",
+                                  "m16n8192k8192_f16_bcol"])
+def test_config_every_element(name):
+    _dense_case(workloads.get(name), sampled=False)
+
+
+@pytest.mark.parametrize("name", ["square4096_bf16", "square4096_f16", "square8192_bf16",
+                                  "square8192_f16", "m4096n4096k512_f16_bcol"])
+def test_config_sampled(name):
+    _dense_case(workloads.get(name), sampled=True)
+
+
+def test_moe_grouped_sampled():
+    w = workloads.get("moe32_m8192n1408k4096_bf16_relu")
+    X, W, rows_per, bias = workloads.make_grouped_inputs(w)
+    total = int(rows_per.sum())
+    dX, dW = X.cuda(), W.cuda()
+    drows = torch.from_numpy(rows_per).cuda()
+    g = Guarded(total, w.N, w.N, torch.bfloat16)
+    rc = dg.grouped_gemm(w.experts, drows, total, w.N, w.K, dX, w.K, dW, w.N, w.K * w.N, g.ptr,
+                         w.N, None, dg.GEMM_EPI_RELU, dg.GEMM_BF16)
+    assert rc == 0, dg.gemm_status_string(rc)
+    torch.cuda.synchronize()
+    assert dg.gemm_device_status() == 0
+    got = g.matrix().double().cpu().numpy()
+    g.check_canaries()
+    r, c = workloads.sample_indices(total, w.N, group_rows=rows_per)
+    ref = oracle.grouped_gemm_at(rows_per, w.N, w.K, X, w.K, W, w.N, w.K * w.N, r, c, relu=True,
+                                 dtype="bf16", threads=THREADS)
+    compare(got[r, c], ref, 2, w.name)
+
+
+# ------------------------------------------------ bit-exact integer cases
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("b_col", [False, True])
+@pytest.mark.parametrize("config", [0, 1])
+def test_exact_integers(dtype, b_col, config):
+    """Integer inputs in [-2, 2] with K <= 4096: every partial sum is an
+    exact integer below 2^24, so the fp32 accumulator is exact in any order
+    and the fp32 output must equal the oracle bit for bit; the 16-bit output
+    must equal the round-to-nearest-even of that exact value."""
+    M, N, K = 300, 520, 1000
+    gen = torch.Generator().manual_seed(77 + config)
+    A = torch.randint(-2, 3, (M, K), generator=gen).to(dtype)
+    B = torch.randint(-2, 3, (N, K) if b_col else (K, N), generator=gen).to(dtype)
+    bias = torch.randint(-4, 5, (N,), generator=gen).to(dtype)
+    ref = oracle.gemm(M, N, K, A, K, B, K if b_col else N, b_colmajor=b_col, bias=bias,
+                      relu=True, dtype=in_name(A), threads=THREADS)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        g32 = run_gemm(A.cuda(), B.cuda(), bias.cuda(), M, N, K, b_col=b_col, relu=True,
+                       out_f32=True)
+        g16 = run_gemm(A.cuda(), B.cuda(), bias.cuda(), M, N, K, b_col=b_col, relu=True)
+    finally:
+        dg.gemm_force_config(-1)
+    got32 = g32.matrix().double().cpu().numpy()
+    assert np.array_equal(got32, ref)
+    expect16 = torch.from_numpy(ref).to(dtype)  # RNE of the exact value
+    assert torch.equal(g16.matrix().cpu(), expect16)
+    g32.check_canaries()
+    g16.check_canaries()
+
+
+# ----------------------------------------------------------- edge cases
+
+@pytest.mark.parametrize("M,N,K", [(1, 1, 1), (7, 9, 5), (130, 200, 72), (129, 257, 65),
+                                   (256, 16, 64), (64, 8, 1000), (3, 4100, 70)])
+@pytest.mark.parametrize("b_col", [False, True])
+def test_ragged_shapes(M, N, K, b_col):
+    gen = torch.Generator().manual_seed(M * 31 + N * 7 + K)
+    A = (torch.rand(M, K, generator=gen) * 2 - 1).half()
+    B = (torch.rand(*((N, K) if b_col else (K, N)), generator=gen) * 2 - 1).half()
+    bias = (torch.rand(N, generator=gen) * 2 - 1).half()
+    # leading dimensions with padding (NaN-filled: any read past the edge shows)
+    lda = (K + 15) // 8 * 8
+    ldb = ((K if b_col else N) + 15) // 8 * 8
+    dA = pad_cols(A.cuda(), lda)
+    dB = pad_cols(B.cuda(), ldb)
+    g = run_gemm(dA, dB, bias.cuda(), M, N, K, b_col=b_col, relu=True, ldc=(N + 23) // 8 * 8)
+    ref = oracle.gemm(M, N, K, A, K, B, K if b_col else N, b_colmajor=b_col, bias=bias,
+                      relu=True, threads=THREADS)
+    compare(g.matrix().double().cpu().numpy(), ref, 2, f"{M}x{N}x{K}")
+    g.check_canaries()
+
+
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_k_zero_writes_act_bias(out_f32):
+    M, N = 37, 50
+    bias = torch.linspace(-3, 3, N).half()
+    g = run_gemm(torch.empty(0, 0, dtype=torch.half, device="cuda"),
+                 torch.empty(0, 0, dtype=torch.half, device="cuda"), bias.cuda(), M, N, 0,
+                 relu=True, out_f32=out_f32)
+    ref = oracle.gemm(M, N, 0, None, 0, None, 0, bias=bias, relu=True)
+    compare(g.matrix().double().cpu().numpy(), ref, 4 if out_f32 else 2, "K=0")
+    g.check_canaries()
+
+
+def test_empty_m_or_n_is_a_noop():
+    g = Guarded(4, 8, 8, torch.float16)
+    A = torch.ones(4, 8, dtype=torch.half, device="cuda")
+    assert dg.gemm(0, 8, 8, A, 8, A, 8, g.ptr, 8, None, 0, dg.GEMM_F16) == 0
+    assert dg.gemm(4, 0, 8, A, 8, A, 8, g.ptr, 8, None, 0, dg.GEMM_F16) == 0
+    torch.cuda.synchronize()
+    assert bool((g.ibuf.cpu() == g.sent).all())
+
+
+@pytest.mark.parametrize("config", range(4))
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_every_config_on_ragged_problem(config, dtype, out_f32):
+    name = dg.gemm_config_name(config)
+    swap = name.startswith("swap")
+    M, N, K = (29 if swap else 333), 712, 328
+    gen = torch.Generator().manual_seed(1000 + config)
+    A = torch.randn(M, K, generator=gen).to(dtype)
+    layouts = [True] if swap else [False, True]
+    for b_col in layouts:
+        B = torch.randn(*((N, K) if b_col else (K, N)), generator=gen).to(dtype)
+        bias = torch.randn(N, generator=gen).to(dtype)
+        ref = oracle.gemm(M, N, K, A, K, B, K if b_col else N, b_colmajor=b_col, bias=bias,
+                          dtype=in_name(A), threads=THREADS)
+        assert dg.gemm_force_config(config) == 0
+        try:
+            g = run_gemm(A.cuda(), B.cuda(), bias.cuda(), M, N, K, b_col=b_col, out_f32=out_f32)
+        finally:
+            dg.gemm_force_config(-1)
+        compare(g.matrix().double().cpu().numpy(), ref, 4 if out_f32 else 2,
+                f"{name} b_col={b_col}")
+        g.check_canaries()
+
+
+def test_swap_config_rejects_row_major_b():
+    n = [i for i in range(dg.gemm_num_configs()) if dg.gemm_config_name(i).startswith("swap")][0]
+    A = torch.ones(16, 64, dtype=torch.half, device="cuda")
+    B = torch.ones(64, 64, dtype=torch.half, device="cuda")
+    C = torch.empty(16, 64, dtype=torch.half, device="cuda")
+    assert dg.gemm_force_config(n) == 0
+    try:
+        assert dg.gemm(16, 64, 64, A, 64, B, 64, C, 64, None, 0,
+                       dg.GEMM_F16) == dg.GEMM_ERR_UNSUPPORTED
+    finally:
+        dg.gemm_force_config(-1)
+
+
+def test_runs_on_a_side_stream():
+    s = torch.cuda.Stream()
+    w = workloads.get("square256_f16")
+    A, B, _ = workloads.make_inputs(w)
+    with torch.cuda.stream(s):
+        dA, dB = A.cuda(), B.cuda()
+        out = dg.matmul(dA, dB, stream=s)
+    s.synchronize()
+    ref = oracle.gemm(256, 256, 256, A, 256, B, 256, threads=THREADS)
+    compare(out.double().cpu().numpy(), ref, 2, "side stream")
+
+
+# --------------------------------------------------------------- grouped
+
+@pytest.mark.parametrize("b_col", [False, True])
+@pytest.mark.parametrize("out_f32", [False, True])
+@pytest.mark.parametrize("config", [0, 1])
+def test_grouped_every_element(b_col, out_f32, config):
+    rows_per = np.array([0, 3, 130, 1, 0, 257, 64, 0], dtype=np.int32)
+    G, N, K = len(rows_per), 200, 136
+    total = int(rows_per.sum())
+    gen = torch.Generator().manual_seed(5 + config)
+    X = torch.randn(total, K, generator=gen).bfloat16()
+    W = (torch.randn(*((G, N, K) if b_col else (G, K, N)), generator=gen) * 0.1).bfloat16()
+    bias = torch.randn(G, N, generator=gen).bfloat16()
+    ref = oracle.grouped_gemm(rows_per, N, K, X, K, W, K if b_col else N, N * K,
+                              b_colmajor=b_col, bias=bias, relu=True, dtype="bf16",
+                              threads=THREADS)
+    dt = torch.float32 if out_f32 else torch.bfloat16
+    ldc = N + 8
+    g = Guarded(total, N, ldc, dt)
+    epi = dg.GEMM_EPI_BIAS | dg.GEMM_EPI_RELU | (dg.GEMM_B_COL_MAJOR if b_col else 0)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        rc = dg.grouped_gemm(G, torch.from_numpy(rows_per).cuda(), total, N, K, X.cuda(), K,
+                             W.cuda(), K if b_col else N, N * K, g.ptr, ldc, bias.cuda(), epi,
+                             dg.GEMM_BF16_OUT_F32 if out_f32 else dg.GEMM_BF16)
+    finally:
+        dg.gemm_force_config(-1)
+    assert rc == 0, dg.gemm_status_string(rc)
+    torch.cuda.synchronize()
+    assert dg.gemm_device_status() == 0
+    compare(g.matrix().double().cpu().numpy(), ref, 4 if out_f32 else 2, "grouped")
+    g.check_canaries()
+
+
+def test_grouped_counts_beyond_total_are_clipped_and_reported():
+    rows_per = np.array([5, 300, 40], dtype=np.int32)  # sums to 345
+    total, N, K = 200, 64, 64                           # caller says 200
+    X = torch.randn(total, K).bfloat16()
+    W = torch.randn(3, K, N).bfloat16()
+    g = Guarded(total, N, N, torch.bfloat16)
+    rc = dg.grouped_gemm(3, torch.from_numpy(rows_per).cuda(), total, N, K, X.cuda(), K,
+                         W.cuda(), N, K * N, g.ptr, N, None, 0, dg.GEMM_BF16)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert dg.gemm_device_status() == dg.GEMM_ERR_INVALID_ARG
+    g.check_canaries()
+    # the rows that exist are still right: group 0 rows 0..4, group 1 rows 5..199
+    ref = oracle.grouped_gemm(np.array([5, 195], dtype=np.int32), N, K, X, K, W, N, K * N,
+                              dtype="bf16", threads=THREADS)
+    compare(g.matrix().double().cpu().numpy(), ref, 2, "clipped groups")
+
+
+# -------------------------------------------------------------- watchdog
+
+def test_watchdog_times_out_cleanly_and_context_survives():
+    assert dg.gemm_watchdog_selftest(2_000_000) == dg.GEMM_ERR_DEVICE_TIMEOUT
+    assert dg.gemm_device_status() == 0  # cleared by the self-test
+    w = workloads.get("square256_f16")
+    A, B, _ = workloads.make_inputs(w)
+    out = dg.matmul(A.cuda(), B.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.gemm(256, 256, 256, A, 256, B, 256, threads=THREADS)
+    compare(out.double().cpu().numpy(), ref, 2, "after watchdog")
