@@ -225,6 +225,8 @@ def bench_ours(args, rank, local, world):
     w = workloads.get(args.workload)
     stream = torch.cuda.current_stream(dev)
     lib = dg.lib()
+    if args.config >= 0 and lib.gemm_force_config(args.config):
+        raise SystemExit(f"unknown config id {args.config}")
 
     if w.grouped:
         X, W, rows, bias = workloads.make_grouped_inputs(w)
@@ -420,6 +422,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--config", type=int, default=-1,
+                    help="force a tile config id (default: the library's table)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (for quick runs)")
     args = ap.parse_args(argv)

@@ -19,6 +19,8 @@ static const Config kConfigs[] = {
     {"tc1_128x128_s6_g8", kKindSingle, 128, 6, 8},
     {"swap_128x16_s8", kKindSwap, 16, 8, 1},
     {"swap_128x32_s8", kKindSwap, 32, 8, 1},
+    {"pair_256x256_s6_g8", kKindPair, 256, 6, 8},
+    {"pair_256x128_s8_g8", kKindPair, 128, 8, 8},
 };
 static constexpr int kNumConfigs = static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0]));
 
@@ -33,6 +35,14 @@ struct Rule {
 
 // BEGIN RULES (written by the sweep)
 static const Rule kRules[] = {
+    {256, 256, 256, 256, 256, 256, 0, 0, 1},  // square256: tc1_128x128_s6_g8 3 TFLOP/s
+    {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 1},  // m1024n1024k2048: tc1_128x128_s6_g8 233 TFLOP/s
+    {2048, 2048, 2048, 2048, 2048, 2048, 0, 0, 0},  // square2048: tc1_128x256_s4_g8 762 TFLOP/s
+    {4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 4},  // square4096: pair_256x256_s6_g8 1266 TFLOP/s
+    {8192, 8192, 8192, 8192, 8192, 8192, 0, 0, 4},  // square8192: pair_256x256_s6_g8 1449 TFLOP/s
+    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 1},  // m1000n1000k2000_bcol: tc1_128x128_s6_g8 196 TFLOP/s
+    {4096, 4096, 4096, 4096, 512, 512, 1, 0, 0},  // m4096n4096k512_bcol: tc1_128x256_s4_g8 559 TFLOP/s
+    {16, 16, 8192, 8192, 8192, 8192, 1, 0, 2},  // m16n8192k8192_bcol: swap_128x16_s8 46 TFLOP/s
     {0, 0, 0, 0, 0, 0, -1, -1, -1},  // sentinel
 };
 // END RULES
@@ -50,6 +60,10 @@ inline int table_lookup(int M, int N, int K, bool b_col, bool grouped) {
   // at least one tile on most SMs.
   if (!grouped && b_col && M <= 32) return M <= 16 ? 2 : 3;
   const long long tiles256 = static_cast<long long>((M + 127) / 128) * ((N + 255) / 256);
+  const long long pair_tiles = static_cast<long long>((M + 255) / 256) * ((N + 255) / 256);
+  // CTA pairs halve the shared-memory operand traffic per MMA, which wins
+  // once every pair gets about two tiles and the K loop is long
+  if (!grouped && pair_tiles >= 128 && K >= 1024) return 4;
   if (N <= 128 || tiles256 < 96) return 1;
   return 0;
 }

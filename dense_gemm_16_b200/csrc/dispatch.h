@@ -14,6 +14,7 @@ struct KernelEntry {
 enum ConfigKind : int {
   kKindSingle = 0,  // one CTA per 128 x BN tile
   kKindSwap = 1,    // skinny problems: C^T = B^T A^T, N fills the MMA rows
+  kKindPair = 2,    // two CTAs (cta_group::2) per 256 x BN tile
 };
 
 struct Config {
@@ -29,5 +30,6 @@ struct Config {
 KernelEntry kernels_bn256(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_bn128(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_swap(int bn, bool bf16, bool out_f32);
+KernelEntry kernels_pair(int bn, bool q_mn, bool bf16, bool out_f32);
 
 }  // namespace dg16

@@ -175,20 +175,33 @@ KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool gro
     if (q_mn || grouped) return {nullptr, 0};  // needs column-major B
     return kernels_swap(c.bn, bf16, f32);
   }
+  if (c.kind == kKindPair) {
+    if (grouped) return {nullptr, 0};
+    return kernels_pair(c.bn, q_mn, bf16, f32);
+  }
   if (c.bn == 256) return kernels_bn256(q_mn, bf16, f32, grouped);
   if (c.bn == 128) return kernels_bn128(q_mn, bf16, f32, grouped);
   return {nullptr, 0};
 }
 
 int launch(const KernelEntry& k, int grid, cudaStream_t stream, const CUtensorMap& tp,
-           const CUtensorMap& tq, const KParams& kp) {
+           const CUtensorMap& tq, const KParams& kp, int cluster = 1) {
   cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = k.smem;
   cfg.stream = stream;
   cfg.attrs = nullptr;
   cfg.numAttrs = 0;
+  if (cluster > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
   void* args[3] = {const_cast<CUtensorMap*>(&tp), const_cast<CUtensorMap*>(&tq),
                    const_cast<KParams*>(&kp)};
   cudaError_t e = cudaLaunchKernelExC(&cfg, k.fn, args);
@@ -277,6 +290,7 @@ int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t
   if (cid < 0 || cid >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
   const Config& cfg = kConfigs[cid];
   const bool swap = cfg.kind == kKindSwap;
+  const bool pair = cfg.kind == kKindPair;
   const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false);
   if (!k.fn || (swap && !bcol)) return GEMM_ERR_UNSUPPORTED;
   rc = ensure_smem_attr(ds, k);
@@ -302,8 +316,10 @@ int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t
     rc = make_map(&tp, A, bf16, 2, dA, &lda_b, bA);
     if (rc) return rc;
     if (bcol) {
+      // the pair kernel's CTAs each load half of the tile's B columns
       const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
-      const uint32_t bB[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn)};
+      const uint32_t bB[2] = {static_cast<uint32_t>(kBK),
+                              static_cast<uint32_t>(pair ? cfg.bn / 2 : cfg.bn)};
       rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
     } else {
       const uint64_t dB[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K)};
@@ -311,7 +327,8 @@ int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t
       rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
     }
     if (rc) return rc;
-    kp.num_p = (M + kBM - 1) / kBM;
+    const int rows_per_tile = pair ? 2 * kBM : kBM;
+    kp.num_p = (M + rows_per_tile - 1) / rows_per_tile;
     kp.num_q = (N + cfg.bn - 1) / cfg.bn;
   } else {
     // P = B stored N x K, Q = A (M x K); the accumulator is C^T
@@ -327,6 +344,10 @@ int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t
     kp.num_q = (M + cfg.bn - 1) / cfg.bn;
   }
   kp.num_tiles = static_cast<long long>(kp.num_p) * kp.num_q;
+  if (pair) {
+    const int pairs = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms / 2));
+    return launch(k, 2 * pairs, stream, tp, tq, kp, 2);
+  }
   const int grid = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms));
   return launch(k, grid, stream, tp, tq, kp);
 }

@@ -29,163 +29,9 @@
 // its tensor memory and returns.
 #pragma once
 
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
-
-#include <type_traits>
-
-#include "ptx.cuh"
-#include "raster.h"
+#include "kernel_common.cuh"
 
 namespace dg16 {
-
-constexpr int kBM = 128;         // MMA rows per CTA
-constexpr int kBK = 64;          // K elements per stage = one 128-byte swizzle row
-constexpr int kThreads = 192;    // 6 warps
-constexpr int kMaxGroups = 1024; // grouped GEMM: groups per launch
-
-// Device status word codes (first error wins).
-enum : unsigned {
-  kStatusOk = 0,
-  kStatusTimeoutProducer = 1,
-  kStatusTimeoutMma = 2,
-  kStatusTimeoutEpilogue = 3,
-  kStatusTimeoutSelftest = 4,
-  kStatusBadGroups = 16,
-};
-
-struct KParams {
-  int M, N, K;            // dense: problem size; grouped: total rows, N, K
-  int num_p, num_q;       // dense tile grid (P blocks x Q blocks)
-  int num_kb;             // K blocks of kBK
-  int group_m;            // raster group height
-  long long num_tiles;    // dense tile count
-  void* C;
-  long long ldc;
-  const void* bias;
-  int epi;                // bit0 bias, bit1 relu
-  const int* group_rows;  // grouped: device counts
-  int num_groups;
-  unsigned* status;       // device status word
-  unsigned long long timeout_ns;
-};
-
-struct SharedCtl {
-  int abort;
-  unsigned tmem_base;
-};
-
-// Bounded wait on an mbarrier phase.  Returns false when the block is
-// aborting (another warp gave up) or when this wait itself ran out, in which
-// case it records `code` and raises the block's abort flag.
-__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, SharedCtl* ctl,
-                                           const KParams& p, unsigned code) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  for (uint32_t n = 1;; ++n) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((n & 63u) == 0) {
-      if (*reinterpret_cast<volatile int*>(&ctl->abort)) return false;
-      if (global_timer_ns() - t0 > p.timeout_ns) {
-        atomicCAS(p.status, 0u, code);
-        *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
-        return false;
-      }
-    }
-  }
-}
-
-// Bounded wait that ignores the abort flag: used only to drain a block's
-// own asynchronous work on the way out.
-__device__ __forceinline__ bool wait_phase_drain(uint32_t bar, uint32_t parity,
-                                                 unsigned long long limit_ns) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity))
-    if (global_timer_ns() - t0 > limit_ns) return false;
-  return true;
-}
-
-template <typename T>
-__device__ __forceinline__ float to_f32(T v);
-template <>
-__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
-template <>
-__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
-  return __bfloat162float(v);
-}
-
-// Pack two fp32 values into the 32-bit pair of the output type (RNE).
-template <typename OutT>
-__device__ __forceinline__ uint32_t pack2(float a, float b);
-template <>
-__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
-  __half2 h = __floats2half2_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-template <>
-__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-  return *reinterpret_cast<uint32_t*>(&h);
-}
-
-template <typename OutT>
-__device__ __forceinline__ OutT from_f32(float v);
-template <>
-__device__ __forceinline__ __half from_f32<__half>(float v) { return __float2half_rn(v); }
-template <>
-__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
-  return __float2bfloat16_rn(v);
-}
-template <>
-__device__ __forceinline__ float from_f32<float>(float v) { return v; }
-
-// Where a tile lives.
-struct TileCoord {
-  int p0;        // first P row (dense: global; grouped: global row of A)
-  int q0;        // first Q row
-  int group;     // grouped: group index (0 otherwise)
-  int row_end;   // grouped: one past the group's last global row
-  bool valid;
-};
-
-// Grouped-GEMM schedule: per-group tile prefix and row starts, in shared memory.
-struct GroupTable {
-  int tile_start[kMaxGroups + 1];
-  int row_start[kMaxGroups + 1];
-};
-
-template <bool GROUPED>
-__device__ __forceinline__ TileCoord tile_coord(long long t, const KParams& p, int num_q_blocks,
-                                                const GroupTable* gt, int& gcursor) {
-  TileCoord c;
-  c.group = 0;
-  c.valid = true;
-  if constexpr (!GROUPED) {
-    int pb, qb;
-    raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
-    c.p0 = pb * kBM;
-    c.q0 = qb;  // caller scales by BN
-    c.row_end = p.M;
-  } else {
-    // tiles are visited in increasing order by each role, so walk forward
-    while (gcursor < p.num_groups && t >= gt->tile_start[gcursor + 1]) ++gcursor;
-    if (gcursor >= p.num_groups) {
-      c.valid = false;
-      return c;
-    }
-    const int g = gcursor;
-    const int local = static_cast<int>(t - gt->tile_start[g]);
-    const int rows = gt->row_start[g + 1] - gt->row_start[g];
-    const int mblocks = (rows + kBM - 1) / kBM;
-    int mb, nb;
-    raster_tile(local, mblocks, num_q_blocks, p.group_m, mb, nb);
-    c.group = g;
-    c.p0 = gt->row_start[g] + mb * kBM;
-    c.q0 = nb;
-    c.row_end = min(gt->row_start[g + 1], p.M);
-  }
-  return c;
-}
 
 // The kernel.
 //   BN      Q rows per tile = MMA N (multiple of 16; of 64 when Q is MN-major)
@@ -405,47 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * BN;
       if constexpr (!SWAP) {
         // accumulator row = output row prow, columns q0 .. q0+BN
-        const bool row_ok = prow < c.row_end;
         const InT* bias_g = has_bias ? bias + static_cast<long long>(c.group) * p.N : nullptr;
-        OutT* crow = C + static_cast<long long>(prow) * p.ldc;
-#pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 32) {
-          const int col0 = q0 + cc;
-          if (col0 >= p.N) break;  // warp-uniform
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(taddr + cc, v);
-          tmem_ld_wait();
-          float f[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            float x = __uint_as_float(v[j]);
-            if (has_bias && col0 + j < p.N) x += to_f32<InT>(bias_g[col0 + j]);
-            if (relu) x = fmaxf(x, 0.0f);
-            f[j] = x;
-          }
-          if (row_ok) {
-            if (col0 + 32 <= p.N) {
-              if constexpr (sizeof(OutT) == 2) {
-                uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                  dst[j] = make_uint4(pack2<OutT>(f[8 * j + 0], f[8 * j + 1]),
-                                      pack2<OutT>(f[8 * j + 2], f[8 * j + 3]),
-                                      pack2<OutT>(f[8 * j + 4], f[8 * j + 5]),
-                                      pack2<OutT>(f[8 * j + 6], f[8 * j + 7]));
-              } else {
-                float4* dst = reinterpret_cast<float4*>(crow + col0);
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                  dst[j] = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
-              }
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (col0 + j < p.N) crow[col0 + j] = from_f32<OutT>(f[j]);
-            }
-          }
-        }
+        store_acc_rows<BN, InT, OutT>(taddr, prow, c.row_end, q0, p, bias_g, relu, C);
       } else {
         // accumulator row = output column prow (an N index); accumulator
         // columns are output rows q0 .. q0+BN

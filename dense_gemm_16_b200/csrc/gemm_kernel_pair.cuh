@@ -1,0 +1,225 @@
+// gemm_kernel_pair.cuh -- the CTA-pair (cta_group::2) variant of the GEMM.
+//
+// Two CTAs on neighbouring SMs (a cluster of 2) share one 256 x BN output
+// tile.  Each CTA streams its own 128 rows of A and its own half (BN/2
+// columns) of B into its own shared memory; the pair's leader issues
+// tcgen05.mma with M = 256, which reads A and B from both CTAs and leaves
+// each CTA's 128 x BN slice of the accumulator in that CTA's tensor memory.
+// Per output element each SM now stages half as much of B as the single-CTA
+// kernel, which halves the shared-memory operand traffic per MMA -- the
+// limit the single-CTA kernel runs into at 128 x 256 tiles.
+//
+// No load is multicast: every CTA fetches its own operand halves.
+//
+// Synchronisation (barriers live in each CTA's shared memory):
+//   full[s]   leader only; armed by the leader's producer with both CTAs'
+//             bytes; both CTAs' TMA copies count their bytes on it.
+//   empty[s]  one per CTA; the leader's MMA thread commits to both.
+//   accf[a]   one per CTA; the leader's MMA thread commits to both.
+//   acce[a]   leader only; one arrival per epilogue warp of either CTA (8).
+#pragma once
+
+#include "kernel_common.cuh"
+
+namespace dg16 {
+
+// BN      output columns per pair tile = MMA N (each CTA loads BN/2 of B)
+// STAGES  ring depth
+// Q_MN    B is row-major (MN-major operand)
+// IN_BF16 / OutT as in the single-CTA kernel
+template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
+                    const KParams p) {
+  using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
+  constexpr int HALF_N = BN / 2;
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair MMA N must be 64..256");
+  static_assert(!Q_MN || HALF_N % 64 == 0, "MN-major B halves are whole 64-column rows");
+  constexpr uint32_t P_BYTES = kBM * kBK * 2;       // this CTA's 128 rows of A
+  constexpr uint32_t Q_BYTES = HALF_N * kBK * 2;    // this CTA's half of B
+  constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
+  constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
+  constexpr uint32_t IDESC = f16_idesc(2 * kBM, BN, IN_BF16 ? 1u : 0u, 0u, Q_MN ? 1u : 0u);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
+  uint8_t* sP = smem;
+  uint8_t* sQ = smem + STAGES * P_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sQ + STAGES * Q_BYTES);
+  uint64_t* full_bar = bars;
+  uint64_t* empty_bar = bars + STAGES;
+  uint64_t* accf_bar = bars + 2 * STAGES;
+  uint64_t* acce_bar = bars + 2 * STAGES + 2;
+  uint64_t* drain_bar = bars + 2 * STAGES + 4;
+  SharedCtl* ctl = reinterpret_cast<SharedCtl*>(bars + 2 * STAGES + 5);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();  // 0 = leader
+  const uint32_t peer = rank ^ 1u;
+  // Every CTA of a pair shares the same smem layout, so a barrier's offset
+  // names the same barrier role in either CTA.
+  const long long pair_id = blockIdx.x >> 1;
+  const long long num_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(smem_u32(&accf_bar[a]), 1);
+      mbar_init(smem_u32(&acce_bar[a]), 2 * 4);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    ctl->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_shared();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmP);
+    tma_prefetch_desc(&tmQ);
+  }
+  if (warp == 1) {
+    tmem_alloc<2>(smem_u32(&ctl->tmem_base), TMEM_COLS);
+    tmem_relinquish<2>();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers are initialised before any remote use
+  tc_fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  const long long num_tiles = p.num_tiles;
+
+  if (warp == 0) {
+    // ---------------------------------------------- TMA producer (both CTAs)
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      uint32_t it = 0;
+      bool ok = true;
+      for (long long t = pair_id; t < num_tiles && ok; t += num_pairs) {
+        int pb, qb;
+        raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
+        const int prow0 = pb * (2 * kBM) + static_cast<int>(rank) * kBM;
+        const int qcol0 = qb * BN + static_cast<int>(rank) * HALF_N;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_phase<true>(smem_u32(&empty_bar[s]), ph ^ 1u, ctl, p, kStatusTimeoutProducer)) {
+            ok = false;
+            break;
+          }
+          // the leader's full barrier counts both CTAs' bytes
+          const uint32_t fb_leader = map_shared_rank(smem_u32(&full_bar[s]), 0);
+          if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * STAGE_BYTES);
+          tma_load_2d_pair(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, prow0, fb_leader, pol);
+          const uint32_t qdst = smem_u32(sQ + s * Q_BYTES);
+          if constexpr (Q_MN) {
+#pragma unroll
+            for (int j = 0; j < HALF_N / 64; ++j)
+              tma_load_2d_pair(qdst + j * (64 * kBK * 2), &tmQ, qcol0 + 64 * j, kb * kBK,
+                               fb_leader, pol);
+          } else {
+            tma_load_2d_pair(qdst, &tmQ, kb * kBK, qcol0, fb_leader, pol);
+          }
+        }
+      }
+      if (!ok) {
+        if (rank == 0) {
+          const uint32_t first = it > STAGES ? it - STAGES : 0;
+          for (uint32_t j = first; j < it; ++j)
+            wait_phase_drain(smem_u32(&full_bar[j % STAGES]), (j / STAGES) & 1u, 50000000ull);
+        }
+        // the peer cannot observe its copies' completion (they count on the
+        // leader's barrier): give any copy in flight time to land
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 2000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------- MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      uint32_t it = 0, local = 0;
+      bool ok = true;
+      const uint32_t peer_empty0 = map_shared_rank(smem_u32(&empty_bar[0]), peer);
+      const uint32_t peer_accf0 = map_shared_rank(smem_u32(&accf_bar[0]), peer);
+      for (long long t = pair_id; t < num_tiles && ok; t += num_pairs, ++local) {
+        const uint32_t a = local & 1u;
+        const uint32_t aph = (local >> 1) & 1u;
+        if (!wait_phase<true>(smem_u32(&acce_bar[a]), aph ^ 1u, ctl, p, kStatusTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + a * BN;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const uint32_t s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1u;
+          if (!wait_phase<true>(smem_u32(&full_bar[s]), ph, ctl, p, kStatusTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t pbase = smem_u32(sP + s * P_BYTES);
+          const uint32_t qbase = smem_u32(sQ + s * Q_BYTES);
+#pragma unroll
+          for (int k = 0; k < kBK / 16; ++k) {
+            const uint64_t adesc = sw128_desc(pbase + k * 32, 16, 1024);
+            const uint64_t bdesc = Q_MN ? sw128_desc(qbase + k * 16 * 128, kBK * 128, 1024)
+                                        : sw128_desc(qbase + k * 32, 16, 1024);
+            mma_f16<2>(d, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          // stage s is free in both CTAs once these MMAs have read it
+          mma_commit<2>(smem_u32(&empty_bar[s]));
+          mma_commit<2>(peer_empty0 + s * 8u);
+        }
+        if (!ok) break;
+        mma_commit<2>(smem_u32(&accf_bar[a]));
+        mma_commit<2>(peer_accf0 + a * 8u);
+      }
+      mma_commit<2>(smem_u32(drain_bar));
+      wait_phase_drain(smem_u32(drain_bar), 0, 50000000ull);
+    }
+    __syncwarp();
+  } else {
+    // --------------------------------------------- epilogue (both CTAs)
+    const int quad = warp & 3;
+    uint32_t local = 0;
+    OutT* C = reinterpret_cast<OutT*>(p.C);
+    const InT* bias = (p.epi & 1) ? reinterpret_cast<const InT*>(p.bias) : nullptr;
+    const bool relu = (p.epi & 2) != 0;
+    const uint32_t acce_leader0 = map_shared_rank(smem_u32(&acce_bar[0]), 0);
+    for (long long t = pair_id; t < num_tiles; t += num_pairs, ++local) {
+      int pb, qb;
+      raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
+      const uint32_t a = local & 1u;
+      const uint32_t aph = (local >> 1) & 1u;
+      const bool ok = wait_phase<true>(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int prow = pb * (2 * kBM) + static_cast<int>(rank) * kBM + quad * 32 + lane;
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * BN;
+      store_acc_rows<BN, InT, OutT>(taddr, prow, p.M, qb * BN, p, bias, relu, C);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce_leader0 + a * 8u);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still signal it
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc<2>(tmem_base, TMEM_COLS);
+  }
+}
+
+template <int BN, int STAGES>
+constexpr int gemm_pair_smem_bytes() {
+  return 1024 + STAGES * (kBM * kBK * 2 + (BN / 2) * kBK * 2) + (2 * STAGES + 5) * 8 +
+         static_cast<int>(sizeof(SharedCtl));
+}
+
+}  // namespace dg16

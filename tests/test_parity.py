@@ -73,7 +73,7 @@ def test_moe_grouped_sampled():
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("b_col", [False, True])
-@pytest.mark.parametrize("config", [0, 1])
+@pytest.mark.parametrize("config", [0, 1, 4, 5])
 def test_exact_integers(dtype, b_col, config):
     """Integer inputs in [-2, 2] with K <= 4096: every partial sum is an
     exact integer below 2^24, so the fp32 accumulator is exact in any order
@@ -144,10 +144,11 @@ def test_empty_m_or_n_is_a_noop():
     assert bool((g.ibuf.cpu() == g.sent).all())
 
 
-@pytest.mark.parametrize("config", range(4))
+@pytest.mark.parametrize("config", range(6))
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("out_f32", [False, True])
 def test_every_config_on_ragged_problem(config, dtype, out_f32):
+    assert config < dg.gemm_num_configs()
     name = dg.gemm_config_name(config)
     swap = name.startswith("swap")
     M, N, K = (29 if swap else 333), 712, 328

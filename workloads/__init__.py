@@ -107,6 +107,8 @@ WORKLOADS = {w.name: w for w in [
        b_colmajor=True),
     _w(name="m16n8192k8192_f16_bcol", M=16, N=8192, K=8192, dtype="f16", seed=10,
        b_colmajor=True),
+    # profiling case: operands (144 MiB) larger than L2, small enough for a full ncu capture
+    _w(name="square6144_bf16", M=6144, N=6144, K=6144, dtype="bf16", dist="normal", seed=12),
     _w(name="moe32_m8192n1408k4096_bf16_relu", M=8192, N=1408, K=4096, dtype="bf16",
        dist="normal", seed=11, relu=True, experts=32, w_std=0.02),
 ]}
