@@ -23,6 +23,9 @@ struct Config {
   int bn;       // MMA N (Q rows per tile)
   int stages;   // operand ring depth
   int group_m;  // raster band height
+  int splits;   // split-K factor (1 = whole K per tile)
+  int pol_p;    // L2 eviction policy of the 128-row operand's copies (kPolicy*)
+  int pol_q;    // ... and of the BN-row operand's copies
 };
 
 // Instances, one getter per translation unit (so they compile in parallel).
@@ -30,6 +33,6 @@ struct Config {
 KernelEntry kernels_bn256(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_bn128(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_swap(int bn, bool bf16, bool out_f32);
-KernelEntry kernels_pair(int bn, bool q_mn, bool bf16, bool out_f32);
+KernelEntry kernels_pair(int bn, int stages, bool q_mn, bool bf16, bool out_f32);
 
 }  // namespace dg16

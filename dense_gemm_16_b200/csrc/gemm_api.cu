@@ -10,7 +10,9 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <algorithm>
 #include <unordered_set>
+#include <vector>
 
 #include "../../include/dense_gemm.h"
 #include "config_table.h"
@@ -61,14 +63,68 @@ struct DeviceState {
 std::mutex g_mu;
 DeviceState g_dev[kMaxDevices];
 
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
 int cuda_fail(cudaError_t e) {
   (void)cudaGetLastError();  // clear a non-sticky error so later calls are unaffected
   (void)e;
   return GEMM_ERR_CUDA;
 }
+
+// Split-K scratch, one buffer per (device, stream): calls on one stream run
+// in order, so they can share it; calls on different streams never do.
+// Layout: [kCounterSlots unsigned counters, zeroed once][partial tiles].
+constexpr size_t kCounterSlots = 65536;
+constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
+struct Workspace {
+  int device;
+  cudaStream_t stream;
+  void* ptr;
+  size_t bytes;
+};
+std::mutex g_ws_mu;
+std::vector<Workspace> g_ws;
+
+// Scratch of at least `partial_bytes` after the counters for (device, stream).
+// The first call per stream allocates (cudaMalloc) and zeroes the counters;
+// a larger request waits for the stream, frees the old buffer and allocates
+// anew.  Kernels leave every counter at 0, so no per-call reset is needed.
+int stream_workspace(int device, cudaStream_t stream, size_t partial_bytes, float** ws,
+                     unsigned** counters) {
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  const size_t need = kCounterBytes + partial_bytes;
+  Workspace* w = nullptr;
+  for (auto& e : g_ws)
+    if (e.device == device && e.stream == stream) w = &e;
+  if (!w || w->bytes < need) {
+    if (w) {
+      cudaError_t e = cudaStreamSynchronize(stream);
+      if (e != cudaSuccess) return cuda_fail(e);
+      cudaFree(w->ptr);
+      w->ptr = nullptr;
+      w->bytes = 0;
+    } else {
+      g_ws.push_back({device, stream, nullptr, 0});
+      w = &g_ws.back();
+    }
+    const size_t bytes = std::max(need, static_cast<size_t>(16) << 20);
+    void* ptr = nullptr;
+    cudaError_t e = cudaMalloc(&ptr, bytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaMemsetAsync(ptr, 0, kCounterBytes, stream);
+    if (e != cudaSuccess) {
+      cudaFree(ptr);
+      return cuda_fail(e);
+    }
+    w->ptr = ptr;
+    w->bytes = bytes;
+  }
+  *counters = static_cast<unsigned*>(w->ptr);
+  *ws = reinterpret_cast<float*>(static_cast<char*>(w->ptr) + kCounterBytes);
+  return GEMM_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
 
 // Device state for the current device, initialised once.
 int device_state(DeviceState** out) {
@@ -177,7 +233,7 @@ KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool gro
   }
   if (c.kind == kKindPair) {
     if (grouped) return {nullptr, 0};
-    return kernels_pair(c.bn, q_mn, bf16, f32);
+    return kernels_pair(c.bn, c.stages, q_mn, bf16, f32);
   }
   if (c.bn == 256) return kernels_bn256(q_mn, bf16, f32, grouped);
   if (c.bn == 128) return kernels_bn128(q_mn, bf16, f32, grouped);
@@ -318,8 +374,10 @@ int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t
     if (bcol) {
       // the pair kernel's CTAs each load half of the tile's B columns
       const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
-      const uint32_t bB[2] = {static_cast<uint32_t>(kBK),
-                              static_cast<uint32_t>(pair ? cfg.bn / 2 : cfg.bn)};
+      // (pair tiles wider than 256 are several N=256 MMAs, each split in two)
+      const uint32_t rows_b = pair ? static_cast<uint32_t>(std::min(cfg.bn, 256) / 2)
+                                   : static_cast<uint32_t>(cfg.bn);
+      const uint32_t bB[2] = {static_cast<uint32_t>(kBK), rows_b};
       rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
     } else {
       const uint64_t dB[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K)};
@@ -344,11 +402,28 @@ int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t
     kp.num_q = (M + cfg.bn - 1) / cfg.bn;
   }
   kp.num_tiles = static_cast<long long>(kp.num_p) * kp.num_q;
+  kp.pol_p = cfg.pol_p;
+  kp.pol_q = cfg.pol_q;
+  kp.splits = 1;
+  kp.kb_per_split = kp.num_kb;
+  if (!pair && cfg.splits > 1 && kp.num_kb >= 2 &&
+      kp.num_tiles <= static_cast<long long>(kCounterSlots)) {
+    const int per = (kp.num_kb + cfg.splits - 1) / cfg.splits;
+    kp.kb_per_split = per;
+    kp.splits = (kp.num_kb + per - 1) / per;  // no empty K range
+    const size_t partial = static_cast<size_t>(kp.num_tiles) * kp.splits * kBM * cfg.bn * 4;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    rc = stream_workspace(dev, stream, partial, &kp.ws, &kp.counters);
+    if (rc) return rc;
+  }
   if (pair) {
     const int pairs = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms / 2));
     return launch(k, 2 * pairs, stream, tp, tq, kp, 2);
   }
-  const int grid = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms));
+  const int grid =
+      static_cast<int>(std::min<long long>(kp.num_tiles * kp.splits, ds->num_sms));
   return launch(k, grid, stream, tp, tq, kp);
 }
 
@@ -437,6 +512,10 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
   kp.num_groups = num_groups;
   kp.status = ds->status;
   kp.timeout_ns = g_timeout_ns.load();
+  kp.pol_p = cfg.pol_p;
+  kp.pol_q = cfg.pol_q;
+  kp.splits = 1;
+  kp.kb_per_split = kp.num_kb;
   // upper bound on tiles: each group adds at most one partial row block
   const long long nq = (N + cfg.bn - 1) / cfg.bn;
   const long long max_tiles = (static_cast<long long>(total_rows) / kBM + num_groups) * nq;

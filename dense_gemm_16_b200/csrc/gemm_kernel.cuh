@@ -129,21 +129,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   long long num_tiles = p.num_tiles;
   if constexpr (GROUPED) num_tiles = gt->tile_start[p.num_groups];
   const int num_q_blocks = GROUPED ? (p.N + BN - 1) / BN : p.num_q;
+  // Work units: (tile, K range).  Without split-K a unit is a whole tile.
+  const int splits = GROUPED ? 1 : p.splits;
+  const int kb_per = splits > 1 ? p.kb_per_split : p.num_kb;
+  const long long num_units = num_tiles * splits;
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
     if (lane == 0) {
-      // A/B panels are re-read by the tiles of the same raster group: keep
-      // them in L2 ahead of the streaming output.
-      const uint64_t pol = policy_evict_last();
+      const uint64_t pol_p = make_policy(p.pol_p);
+      const uint64_t pol_q = make_policy(p.pol_q);
       uint32_t it = 0;
       int gcur = 0;
       bool ok = true;
-      for (long long t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+      for (long long u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
+        const long long t = u / splits;
+        const int kb0 = static_cast<int>(u % splits) * kb_per;
+        const int kb1 = min(kb0 + kb_per, p.num_kb);
         const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
         if (!c.valid) break;
         const int q0 = c.q0 * BN;
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_phase(smem_u32(&empty_bar[s]), ph ^ 1u, ctl, p, kStatusTimeoutProducer)) {
@@ -152,24 +158,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t fb = smem_u32(&full_bar[s]);
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          tma_load_2d(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, c.p0, fb, pol);
+          tma_load_2d(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, c.p0, fb, pol_p);
           const uint32_t qdst = smem_u32(sQ + s * Q_BYTES);
           if constexpr (GROUPED) {
             if constexpr (Q_MN) {
 #pragma unroll
               for (int j = 0; j < BN / 64; ++j)
                 tma_load_3d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, c.group, fb,
-                            pol);
+                            pol_q);
             } else {
-              tma_load_3d(qdst, &tmQ, kb * kBK, q0, c.group, fb, pol);
+              tma_load_3d(qdst, &tmQ, kb * kBK, q0, c.group, fb, pol_q);
             }
           } else {
             if constexpr (Q_MN) {
 #pragma unroll
               for (int j = 0; j < BN / 64; ++j)
-                tma_load_2d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, fb, pol);
+                tma_load_2d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, fb, pol_q);
             } else {
-              tma_load_2d(qdst, &tmQ, kb * kBK, q0, fb, pol);
+              tma_load_2d(qdst, &tmQ, kb * kBK, q0, fb, pol_q);
             }
           }
         }
@@ -188,7 +194,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, local = 0;
       int gcur = 0;
       bool ok = true;
-      for (long long t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++local) {
+      for (long long u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++local) {
+        const long long t = u / splits;
+        const int kb0 = static_cast<int>(u % splits) * kb_per;
+        const int kb1 = min(kb0 + kb_per, p.num_kb);
         const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
         if (!c.valid) break;
         const uint32_t a = local & 1u;
@@ -196,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!wait_phase(smem_u32(&acce_bar[a]), aph ^ 1u, ctl, p, kStatusTimeoutMma)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + a * BN;
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_phase(smem_u32(&full_bar[s]), ph, ctl, p, kStatusTimeoutMma)) {
@@ -215,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // kBK rows apart; 8-row K groups 1024 B apart.
             const uint64_t bdesc = Q_MN ? sw128_desc(qbase + k * 16 * 128, kBK * 128, 1024)
                                         : sw128_desc(qbase + k * 32, 16, 1024);
-            mma_f16<1>(d, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
+            mma_f16<1>(d, adesc, bdesc, IDESC, (kb != kb0 || k != 0) ? 1u : 0u);
           }
           mma_commit<1>(smem_u32(&empty_bar[s]));  // frees the stage when read
         }
@@ -230,13 +239,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ----------------------------------------------------------- epilogue
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
+    const int row_local = quad * 32 + lane;
     uint32_t local = 0;
     int gcur = 0;
     OutT* C = reinterpret_cast<OutT*>(p.C);
     const InT* bias = reinterpret_cast<const InT*>(p.bias);
     const bool has_bias = (p.epi & 1) != 0;
     const bool relu = (p.epi & 2) != 0;
-    for (long long t = blockIdx.x; t < num_tiles; t += gridDim.x, ++local) {
+    for (long long u = blockIdx.x; u < num_units; u += gridDim.x, ++local) {
+      const long long t = u / splits;
+      const int split = static_cast<int>(u % splits);
       const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
       if (!c.valid) break;
       const uint32_t a = local & 1u;
@@ -244,11 +256,75 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every lane waits; the warp proceeds only if all saw the phase, so the
       // .sync.aligned TMEM loads below are always issued by the whole warp
       const bool ok = wait_phase(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (splits > 1) {
+        // the split-K path below syncs the four epilogue warps, so they must
+        // agree on leaving: a failed wait always raises the abort flag first
+        epilogue_bar();
+        if (*reinterpret_cast<volatile int*>(&ctl->abort)) break;
+      } else if (!__all_sync(0xffffffffu, ok)) {
+        break;
+      }
       tc_fence_after();
-      const int prow = c.p0 + quad * 32 + lane;  // this thread's accumulator row
+      const int prow = c.p0 + row_local;  // this thread's accumulator row
       const int q0 = c.q0 * BN;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * BN;
+      if (splits > 1) {
+        // ---- split-K: park this K range's partial tile, the last range sums
+        float* part = p.ws + (t * splits + split) * static_cast<long long>(kBM * BN) +
+                      static_cast<long long>(row_local) * BN;
+#pragma unroll 1
+        for (int cc = 0; cc < BN; cc += 16) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(taddr + cc, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            __stcg(reinterpret_cast<float4*>(part + cc) + j,
+                   make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acce_bar[a]));  // the accumulator is free again
+        __threadfence();
+        epilogue_bar();
+        if (row_local == 0) {
+          const unsigned old = atomicAdd(&p.counters[t], 1u);
+          ctl->last = (old == static_cast<unsigned>(splits - 1)) ? 1 : 0;
+        }
+        epilogue_bar();
+        if (ctl->last) {
+          __threadfence();
+          const float* base = p.ws + t * splits * static_cast<long long>(kBM * BN) +
+                              static_cast<long long>(row_local) * BN;
+          if constexpr (!SWAP) {
+            const InT* bias_g = has_bias ? bias : nullptr;
+            store_partial_sums<BN, InT, OutT>(base, splits, prow, c.row_end, q0, p, bias_g,
+                                              relu, C);
+          } else {
+            const bool col_ok = prow < p.N;
+            const float b = (has_bias && col_ok) ? to_f32<InT>(bias[prow]) : 0.0f;
+#pragma unroll 1
+            for (int cc = 0; cc < BN; cc += 16) {
+              const int row0 = q0 + cc;
+              if (row0 >= p.M) break;
+              float f[16];
+              sum_partials16(base + cc, splits, static_cast<long long>(kBM * BN), f);
+              if (col_ok) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  if (row0 + j < p.M) {
+                    float x = f[j] + b;
+                    if (relu) x = fmaxf(x, 0.0f);
+                    C[static_cast<long long>(row0 + j) * p.ldc + prow] = from_f32<OutT>(x);
+                  }
+                }
+              }
+            }
+          }
+          if (row_local == 0) p.counters[t] = 0u;  // ready for the next launch
+        }
+        continue;
+      }
       if constexpr (!SWAP) {
         // accumulator row = output row prow, columns q0 .. q0+BN
         const InT* bias_g = has_bias ? bias + static_cast<long long>(c.group) * p.N : nullptr;

@@ -23,22 +23,30 @@
 
 namespace dg16 {
 
-// BN      output columns per pair tile = MMA N (each CTA loads BN/2 of B)
+// BN      MMA N (each CTA loads BN/2 columns of B per MMA)
+// NSUB    MMAs per K step, side by side in N: the pair tile is 256 x (BN*NSUB).
+//         With NSUB = 2 and BN = 256 one accumulator fills all 512 TMEM
+//         columns (no double buffering) but each SM stages 25% fewer operand
+//         bytes per FLOP and the ring holds more time's worth of work.
 // STAGES  ring depth
 // Q_MN    B is row-major (MN-major operand)
 // IN_BF16 / OutT as in the single-CTA kernel
-template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT>
+template <int BN, int NSUB, int STAGES, bool Q_MN, bool IN_BF16, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                     const KParams p) {
   using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
   constexpr int HALF_N = BN / 2;
+  constexpr int TILE_N = BN * NSUB;                 // output columns per pair tile
+  constexpr int ACC_BUFS = (2 * TILE_N <= 512) ? 2 : 1;
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "pair MMA N must be 64..256");
+  static_assert(TILE_N <= 512, "the accumulator must fit in 512 TMEM columns");
   static_assert(!Q_MN || HALF_N % 64 == 0, "MN-major B halves are whole 64-column rows");
-  constexpr uint32_t P_BYTES = kBM * kBK * 2;       // this CTA's 128 rows of A
-  constexpr uint32_t Q_BYTES = HALF_N * kBK * 2;    // this CTA's half of B
+  constexpr uint32_t P_BYTES = kBM * kBK * 2;              // this CTA's 128 rows of A
+  constexpr uint32_t QSUB_BYTES = HALF_N * kBK * 2;        // its half of one MMA's B
+  constexpr uint32_t Q_BYTES = NSUB * QSUB_BYTES;
   constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
-  constexpr uint32_t TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
+  constexpr uint32_t TMEM_COLS = (ACC_BUFS * TILE_N <= 256) ? 256 : 512;
   constexpr uint32_t IDESC = f16_idesc(2 * kBM, BN, IN_BF16 ? 1u : 0u, 0u, Q_MN ? 1u : 0u);
 
   extern __shared__ uint8_t smem_raw[];
@@ -95,14 +103,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (both CTAs)
     if (lane == 0) {
-      const uint64_t pol = policy_evict_last();
+      const uint64_t pol_p = make_policy(p.pol_p);
+      const uint64_t pol_q = make_policy(p.pol_q);
       uint32_t it = 0;
       bool ok = true;
       for (long long t = pair_id; t < num_tiles && ok; t += num_pairs) {
         int pb, qb;
         raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
         const int prow0 = pb * (2 * kBM) + static_cast<int>(rank) * kBM;
-        const int qcol0 = qb * BN + static_cast<int>(rank) * HALF_N;
+        // MMA j of the K step covers tile columns [j*BN, (j+1)*BN); this CTA
+        // supplies the rank-th half of each
+        const int qcol0 = qb * TILE_N + static_cast<int>(rank) * HALF_N;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -113,15 +124,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the leader's full barrier counts both CTAs' bytes
           const uint32_t fb_leader = map_shared_rank(smem_u32(&full_bar[s]), 0);
           if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * STAGE_BYTES);
-          tma_load_2d_pair(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, prow0, fb_leader, pol);
-          const uint32_t qdst = smem_u32(sQ + s * Q_BYTES);
-          if constexpr (Q_MN) {
+          tma_load_2d_pair(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, prow0, fb_leader, pol_p);
 #pragma unroll
-            for (int j = 0; j < HALF_N / 64; ++j)
-              tma_load_2d_pair(qdst + j * (64 * kBK * 2), &tmQ, qcol0 + 64 * j, kb * kBK,
-                               fb_leader, pol);
-          } else {
-            tma_load_2d_pair(qdst, &tmQ, kb * kBK, qcol0, fb_leader, pol);
+          for (int sub = 0; sub < NSUB; ++sub) {
+            const uint32_t qdst = smem_u32(sQ + s * Q_BYTES + sub * QSUB_BYTES);
+            const int qc = qcol0 + sub * BN;
+            if constexpr (Q_MN) {
+#pragma unroll
+              for (int j = 0; j < HALF_N / 64; ++j)
+                tma_load_2d_pair(qdst + j * (64 * kBK * 2), &tmQ, qc + 64 * j, kb * kBK,
+                                 fb_leader, pol_q);
+            } else {
+              tma_load_2d_pair(qdst, &tmQ, kb * kBK, qc, fb_leader, pol_q);
+            }
           }
         }
       }
@@ -147,11 +162,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t peer_empty0 = map_shared_rank(smem_u32(&empty_bar[0]), peer);
       const uint32_t peer_accf0 = map_shared_rank(smem_u32(&accf_bar[0]), peer);
       for (long long t = pair_id; t < num_tiles && ok; t += num_pairs, ++local) {
-        const uint32_t a = local & 1u;
-        const uint32_t aph = (local >> 1) & 1u;
+        const uint32_t a = ACC_BUFS == 2 ? (local & 1u) : 0u;
+        const uint32_t aph = ACC_BUFS == 2 ? ((local >> 1) & 1u) : (local & 1u);
         if (!wait_phase<true>(smem_u32(&acce_bar[a]), aph ^ 1u, ctl, p, kStatusTimeoutMma)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + a * BN;
+        const uint32_t d = tmem_base + a * TILE_N;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -165,9 +180,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < kBK / 16; ++k) {
             const uint64_t adesc = sw128_desc(pbase + k * 32, 16, 1024);
-            const uint64_t bdesc = Q_MN ? sw128_desc(qbase + k * 16 * 128, kBK * 128, 1024)
-                                        : sw128_desc(qbase + k * 32, 16, 1024);
-            mma_f16<2>(d, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
+#pragma unroll
+            for (int sub = 0; sub < NSUB; ++sub) {
+              const uint32_t qb_addr = qbase + sub * QSUB_BYTES;
+              const uint64_t bdesc = Q_MN ? sw128_desc(qb_addr + k * 16 * 128, kBK * 128, 1024)
+                                          : sw128_desc(qb_addr + k * 32, 16, 1024);
+              mma_f16<2>(d + sub * BN, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
+            }
           }
           // stage s is free in both CTAs once these MMAs have read it
           mma_commit<2>(smem_u32(&empty_bar[s]));
@@ -192,14 +211,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (long long t = pair_id; t < num_tiles; t += num_pairs, ++local) {
       int pb, qb;
       raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
-      const uint32_t a = local & 1u;
-      const uint32_t aph = (local >> 1) & 1u;
+      const uint32_t a = ACC_BUFS == 2 ? (local & 1u) : 0u;
+      const uint32_t aph = ACC_BUFS == 2 ? ((local >> 1) & 1u) : (local & 1u);
       const bool ok = wait_phase<true>(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const int prow = pb * (2 * kBM) + static_cast<int>(rank) * kBM + quad * 32 + lane;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * BN;
-      store_acc_rows<BN, InT, OutT>(taddr, prow, p.M, qb * BN, p, bias, relu, C);
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * TILE_N;
+      store_acc_rows<TILE_N, InT, OutT>(taddr, prow, p.M, qb * TILE_N, p, bias, relu, C);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader0 + a * 8u);
@@ -216,9 +235,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int BN, int STAGES>
+template <int BN, int NSUB, int STAGES>
 constexpr int gemm_pair_smem_bytes() {
-  return 1024 + STAGES * (kBM * kBK * 2 + (BN / 2) * kBK * 2) + (2 * STAGES + 5) * 8 +
+  return 1024 + STAGES * (kBM * kBK * 2 + NSUB * (BN / 2) * kBK * 2) + (2 * STAGES + 5) * 8 +
          static_cast<int>(sizeof(SharedCtl));
 }
 

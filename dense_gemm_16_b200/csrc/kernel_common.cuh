@@ -43,11 +43,32 @@ struct KParams {
   int num_groups;
   unsigned* status;       // device status word
   unsigned long long timeout_ns;
+  int pol_p, pol_q;       // L2 policy of the P / Q operand copies (kPolicy*)
+  // split-K: each tile's K blocks are cut into `splits` ranges of kb_per_split
+  // blocks; partial fp32 tiles go to `ws` and the last range to finish sums
+  // them (in range order) and runs the epilogue.  splits == 1: no split.
+  int splits, kb_per_split;
+  float* ws;              // [tile][split][128][BN] fp32 partials
+  unsigned* counters;     // [tile] arrivals, left at 0 after every launch
 };
+
+enum : int { kPolicyNormal = 0, kPolicyFirst = 1, kPolicyLast = 2 };
+
+__device__ __forceinline__ uint64_t make_policy(int code) {
+  return code == kPolicyLast ? policy_evict_last()
+         : code == kPolicyFirst ? policy_evict_first() : policy_evict_normal();
+}
+
+// Barrier among the four epilogue warps only (named barrier 1).
+__device__ __forceinline__ void epilogue_bar() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
 
 struct SharedCtl {
   int abort;
   unsigned tmem_base;
+  int last;  // split-K: this block finishes the current tile
+  int pad;
 };
 
 // Bounded wait on an mbarrier phase.  Returns false when the block is
@@ -215,6 +236,70 @@ __device__ __forceinline__ void store_acc_rows(uint32_t taddr, int prow, int row
         for (int j = 0; j < 32; ++j)
           if (col0 + j < p.N) crow[col0 + j] = from_f32<OutT>(f[j]);
       }
+    }
+  }
+}
+
+// Sum of 16 consecutive fp32 values over `splits` partial tiles `stride`
+// floats apart, in split order (so the result does not depend on which
+// block finished last).
+__device__ __forceinline__ void sum_partials16(const float* src, int splits, long long stride,
+                                               float (&f)[16]) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) f[j] = 0.0f;
+  for (int s = 0; s < splits; ++s) {
+    const float4* q = reinterpret_cast<const float4*>(src + s * stride);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 v = __ldcg(q + j);
+      f[4 * j] += v.x;
+      f[4 * j + 1] += v.y;
+      f[4 * j + 2] += v.z;
+      f[4 * j + 3] += v.w;
+    }
+  }
+}
+
+// Split-K finish for one output row: sum the partial rows (row-major
+// [split][128][BN] fp32 starting at `base` for this row), then bias, ReLU,
+// cast and store exactly like store_acc_rows.
+template <int BN, typename InT, typename OutT>
+__device__ __forceinline__ void store_partial_sums(const float* base, int splits, int prow,
+                                                   int row_end, int q0, const KParams& p,
+                                                   const InT* bias_g, bool relu, OutT* C) {
+  const bool row_ok = prow < row_end;
+  OutT* crow = C + static_cast<long long>(prow) * p.ldc;
+  const long long stride = static_cast<long long>(kBM) * BN;
+#pragma unroll 1
+  for (int cc = 0; cc < BN; cc += 16) {
+    const int col0 = q0 + cc;
+    if (col0 >= p.N || !row_ok) break;
+    float f[16];
+    sum_partials16(base + cc, splits, stride, f);
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (bias_g != nullptr && col0 + j < p.N) f[j] += to_f32<InT>(bias_g[col0 + j]);
+      if (relu) f[j] = fmaxf(f[j], 0.0f);
+    }
+    if (col0 + 16 <= p.N) {
+      if constexpr (sizeof(OutT) == 2) {
+        uint4* dst = reinterpret_cast<uint4*>(crow + col0);
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+          dst[j] = make_uint4(pack2<OutT>(f[8 * j + 0], f[8 * j + 1]),
+                              pack2<OutT>(f[8 * j + 2], f[8 * j + 3]),
+                              pack2<OutT>(f[8 * j + 4], f[8 * j + 5]),
+                              pack2<OutT>(f[8 * j + 6], f[8 * j + 7]));
+      } else {
+        float4* dst = reinterpret_cast<float4*>(crow + col0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          dst[j] = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (col0 + j < p.N) crow[col0 + j] = from_f32<OutT>(f[j]);
     }
   }
 }

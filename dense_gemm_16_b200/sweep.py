@@ -5,11 +5,14 @@ The counterpart of the pages' compile-time parameter search ("用Triton跨芯片
 优化GEMM" section 3.3; the crowd-sourced tuning page, sections 3.2 and 5.2):
 enumerate the candidates (here: the configs compiled into the library, already
 pruned by the shared-memory budget when they were instantiated), time each
-with an L2 flush before every repetition, take the median of several batches,
+with an L2 flush before every repetition, interleaving the candidates in
+several rounds so that clock and temperature drift hit them alike, take the
+median,
 keep the fastest, and record every candidate's time -- failures included --
 in a log.
 
-    python -m dense_gemm_16_b200.sweep [--write] [--log PATH] [--reps R] [--batches B]
+    python -m dense_gemm_16_b200.sweep [--write] [--log PATH] [--reps R] [--rounds N]
+                                      [--only CLASS ...]
 
 Needs a GPU.  --write rewrites the RULES block of csrc/config_table.h; the
 library must then be rebuilt.
@@ -41,7 +44,47 @@ CLASSES = [
 ]
 
 
-def _time_config(dg, torch, cid, M, N, K, dtype, b_col, reps, batches, flush):
+def _bench_rounds(dg, torch, calls, reps, rounds, flush):
+    """Time every candidate in `calls` ({config id: launch fn}) `rounds` times,
+    interleaved (so clock and thermal drift hit all candidates alike): each
+    round runs `reps` launches per candidate, L2 flushed before each, and
+    keeps the median; the result per candidate is the median over rounds."""
+    lib = dg.lib()
+    per = {cid: [] for cid in calls}
+    errors = {}
+    for cid, call in list(calls.items()):  # one checked launch each
+        lib.gemm_force_config(cid)
+        try:
+            rc = call()
+            torch.cuda.synchronize()
+            st = dg.gemm_device_status()
+        finally:
+            lib.gemm_force_config(-1)
+        if rc or st:
+            errors[cid] = dg.gemm_status_string(rc or st)
+            del calls[cid]
+    for _ in range(rounds):
+        for cid, call in calls.items():
+            lib.gemm_force_config(cid)
+            try:
+                ts = []
+                for _ in range(reps):
+                    if flush is not None:
+                        flush.fill_(1)
+                    s = torch.cuda.Event(enable_timing=True)
+                    e = torch.cuda.Event(enable_timing=True)
+                    s.record()
+                    call()
+                    e.record()
+                    ts.append((s, e))
+                torch.cuda.synchronize()
+            finally:
+                lib.gemm_force_config(-1)
+            per[cid].append(statistics.median(a.elapsed_time(b) for a, b in ts))
+    return {cid: statistics.median(v) for cid, v in per.items() if v}, errors
+
+
+def _dense_calls(dg, torch, names, M, N, K, dtype, b_col):
     lib = dg.lib()
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
     A = torch.randn(M, K, device="cuda", dtype=tdt)
@@ -51,63 +94,86 @@ def _time_config(dg, torch, cid, M, N, K, dtype, b_col, reps, batches, flush):
     epi = dg.GEMM_B_COL_MAJOR if b_col else 0
     ldb = K if b_col else N
     stream = torch.cuda.current_stream().cuda_stream
-    if lib.gemm_force_config(cid):
-        return None, "bad id"
-    try:
-        def call():
-            return lib.gemm(M, N, K, A.data_ptr(), K, B.data_ptr(), ldb, C.data_ptr(), N, None,
-                            epi, code, stream)
-        rc = call()
-        if rc:
-            return None, dg.gemm_status_string(rc)
-        for _ in range(3):
-            call()
-        torch.cuda.synchronize()
-        if dg.gemm_device_status():
-            return None, "device status"
-        meds = []
-        for _ in range(batches):
-            ts = []
-            for _ in range(reps):
-                flush.fill_(1)
-                s = torch.cuda.Event(enable_timing=True)
-                e = torch.cuda.Event(enable_timing=True)
-                s.record()
-                call()
-                e.record()
-                ts.append((s, e))
-            torch.cuda.synchronize()
-            meds.append(statistics.median(a.elapsed_time(b) for a, b in ts))
-        return statistics.median(meds), ""
-    finally:
-        lib.gemm_force_config(-1)
+    keep = (A, B, C)
+
+    def make():
+        return lambda: lib.gemm(M, N, K, keep[0].data_ptr(), K, keep[1].data_ptr(), ldb,
+                                keep[2].data_ptr(), N, None, epi, code, stream)
+    calls, skipped = {}, {}
+    for cid, name in enumerate(names):
+        if name.startswith("swap") and not b_col:
+            skipped[cid] = "needs column-major B"
+        else:
+            calls[cid] = make()
+    return calls, skipped, keep
 
 
-def run(reps=20, batches=3, log=None):
+# Grouped classes: (name, experts, total rows, N, K, dtype) with the seeded
+# Dirichlet/multinomial routing of the MoE workload.
+GROUPED_CLASSES = [
+    ("moe32_n1408_k4096", 32, 8192, 1408, 4096, "bf16"),
+]
+
+
+def _grouped_calls(dg, torch, names, E, R, N, K, dtype):
+    import workloads
+    lib = dg.lib()
+    rows = workloads.moe_group_rows(E, R, 11)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    X = torch.randn(R, K, device="cuda", dtype=tdt)
+    W = torch.randn(E, K, N, device="cuda", dtype=tdt) * 0.02
+    Y = torch.empty(R, N, device="cuda", dtype=tdt)
+    drows = torch.from_numpy(rows).cuda()
+    code = dg.dtype_code(tdt)
+    stream = torch.cuda.current_stream().cuda_stream
+    keep = (X, W, Y, drows)
+
+    def call():
+        return lib.grouped_gemm(E, keep[3].data_ptr(), R, N, K, keep[0].data_ptr(), K,
+                                keep[1].data_ptr(), N, K * N, keep[2].data_ptr(), N, None,
+                                dg.GEMM_EPI_RELU, code, stream)
+    calls, skipped = {}, {}
+    for cid, name in enumerate(names):
+        if name.startswith(("swap", "pair")) or "_k" in name:
+            skipped[cid] = "not a grouped kernel (or split-K, which grouped ignores)"
+        else:
+            calls[cid] = call
+    return calls, skipped, keep
+
+
+def run(reps=10, rounds=5, log=None, only=None, sustained=False):
+    """sustained=True: launches back to back without the L2 flush, the regime
+    of a long run under the power cap (use inputs larger than L2)."""
     import torch
 
     import dense_gemm_16_b200 as dg
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32, device="cuda")
+    flush = None if sustained else torch.empty(256 * 1024 * 1024 // 4, dtype=torch.int32,
+                                               device="cuda")
     names = [dg.gemm_config_name(i) for i in range(dg.gemm_num_configs())]
     results = []
-    for cname, M, N, K, dtype, b_col in CLASSES:
+    jobs = [(c[0], False, c) for c in CLASSES] + [(c[0], True, c) for c in GROUPED_CLASSES]
+    for cname, grouped, spec in jobs:
+        if only and cname not in only:
+            continue
+        if grouped:
+            _, E, R, N, K, dtype = spec
+            M, b_col = R, False
+            calls, skipped, keep = _grouped_calls(dg, torch, names, E, R, N, K, dtype)
+        else:
+            _, M, N, K, dtype, b_col = spec
+            calls, skipped, keep = _dense_calls(dg, torch, names, M, N, K, dtype, b_col)
+        times, errors = _bench_rounds(dg, torch, calls, reps, rounds, flush)
+        errors.update(skipped)
         row = {"class": cname, "M": M, "N": N, "K": K, "dtype": dtype, "b_col": b_col,
-               "times_ms": {}, "errors": {}}
-        for cid, name in enumerate(names):
-            if name.startswith("swap") and not b_col:
-                row["errors"][name] = "needs column-major B"
-                continue
-            t, err = _time_config(dg, torch, cid, M, N, K, dtype, b_col, reps, batches, flush)
-            if t is None:
-                row["errors"][name] = err
-            else:
-                row["times_ms"][name] = t
-        best = min(row["times_ms"], key=row["times_ms"].get)
-        row["best"] = best
-        row["best_id"] = names.index(best)
-        row["best_tflops"] = 2.0 * M * N * K / (row["times_ms"][best] * 1e-3) / 1e12
+               "grouped": grouped, "times_ms": {names[c]: t for c, t in times.items()},
+               "errors": {names[c]: e for c, e in errors.items()}}
+        best = min(times, key=times.get)
+        row["best"] = names[best]
+        row["best_id"] = best
+        row["best_tflops"] = 2.0 * M * N * K / (times[best] * 1e-3) / 1e12
         results.append(row)
         print(json.dumps(row), flush=True)
+        del keep
     if log:
         with open(log, "w") as f:
             for r in results:
@@ -121,7 +187,8 @@ def write_rules(results, path=TABLE):
     for r in results:
         lines.append(
             f"    {{{r['M']}, {r['M']}, {r['N']}, {r['N']}, {r['K']}, {r['K']}, "
-            f"{int(r['b_col'])}, 0, {r['best_id']}}},  // {r['class']}: {r['best']} "
+            f"{int(r['b_col'])}, {int(r.get('grouped', False))}, {r['best_id']}}},  "
+            f"// {r['class']}: {r['best']} "
             f"{r['best_tflops']:.0f} TFLOP/s")
     lines.append("    {0, 0, 0, 0, 0, 0, -1, -1, -1},  // sentinel")
     lines.append("};")
@@ -134,13 +201,16 @@ def write_rules(results, path=TABLE):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--reps", type=int, default=20)
-    ap.add_argument("--batches", type=int, default=3)
+    ap.add_argument("--reps", type=int, default=10)
+    ap.add_argument("--rounds", type=int, default=5)
     ap.add_argument("--log", default=None)
+    ap.add_argument("--only", nargs="*", default=None, help="class names to sweep")
+    ap.add_argument("--sustained", action="store_true",
+                    help="back-to-back launches, no L2 flush")
     ap.add_argument("--write", action="store_true")
     a = ap.parse_args(argv)
     sys.path.insert(0, ROOT)
-    res = run(a.reps, a.batches, a.log)
+    res = run(a.reps, a.rounds, a.log, a.only, a.sustained)
     if a.write:
         write_rules(res)
 

@@ -73,7 +73,7 @@ def test_moe_grouped_sampled():
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("b_col", [False, True])
-@pytest.mark.parametrize("config", [0, 1, 4, 5])
+@pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 18])
 def test_exact_integers(dtype, b_col, config):
     """Integer inputs in [-2, 2] with K <= 4096: every partial sum is an
     exact integer below 2^24, so the fp32 accumulator is exact in any order
@@ -144,7 +144,7 @@ def test_empty_m_or_n_is_a_noop():
     assert bool((g.ibuf.cpu() == g.sent).all())
 
 
-@pytest.mark.parametrize("config", range(6))
+@pytest.mark.parametrize("config", range(21))
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("out_f32", [False, True])
 def test_every_config_on_ragged_problem(config, dtype, out_f32):
@@ -258,3 +258,57 @@ def test_watchdog_times_out_cleanly_and_context_survives():
     torch.cuda.synchronize()
     ref = oracle.gemm(256, 256, 256, A, 256, B, 256, threads=THREADS)
     compare(out.double().cpu().numpy(), ref, 2, "after watchdog")
+
+
+# --------------------------------------------------------------- split-K
+
+def _split_configs():
+    return [i for i in range(dg.gemm_num_configs()) if "_k" in dg.gemm_config_name(i)]
+
+
+@pytest.mark.parametrize("swap", [False, True])
+def test_split_k_is_deterministic_and_reusable(swap):
+    """Partial tiles are summed in split order by whichever block finishes a
+    tile last, so repeated runs are bit-identical; the arrival counters are
+    left at zero, so a second launch on the same stream is right too."""
+    cfgs = [i for i in _split_configs() if dg.gemm_config_name(i).startswith("swap") == swap]
+    M, N, K = (16, 4096, 4096) if swap else (512, 640, 4096)
+    gen = torch.Generator().manual_seed(31)
+    A = torch.randn(M, K, generator=gen).half()
+    B = torch.randn(N, K, generator=gen).half()
+    ref = oracle.gemm_at(M, N, K, A, K, B, K, *workloads.sample_indices(M, N, n=2048),
+                         b_colmajor=True, threads=THREADS)
+    rows, cols = workloads.sample_indices(M, N, n=2048)
+    for cid in cfgs:
+        assert dg.gemm_force_config(cid) == 0
+        try:
+            outs = [run_gemm(A.cuda(), B.cuda(), None, M, N, K, b_col=True) for _ in range(3)]
+        finally:
+            dg.gemm_force_config(-1)
+        first = outs[0].matrix().cpu()
+        for g in outs[1:]:
+            assert torch.equal(g.matrix().cpu(), first)
+        compare(first.double().numpy()[rows, cols], ref, 2, dg.gemm_config_name(cid))
+
+
+def test_split_k_on_concurrent_streams():
+    cid = [i for i in _split_configs() if dg.gemm_config_name(i).startswith("tc1")][0]
+    M, N, K = 384, 512, 2048
+    gen = torch.Generator().manual_seed(41)
+    As = [torch.randn(M, K, generator=gen).half() for _ in range(3)]
+    B = torch.randn(K, N, generator=gen).half()
+    dB = B.cuda()
+    streams = [torch.cuda.Stream() for _ in range(3)]
+    outs = []
+    assert dg.gemm_force_config(cid) == 0
+    try:
+        for A, s in zip(As, streams):
+            with torch.cuda.stream(s):
+                dA = A.cuda()
+                outs.append(dg.matmul(dA, dB, stream=s))
+        torch.cuda.synchronize()
+    finally:
+        dg.gemm_force_config(-1)
+    for A, o in zip(As, outs):
+        ref = oracle.gemm(M, N, K, A, K, B, N, threads=THREADS)
+        compare(o.double().cpu().numpy(), ref, 2, "split-K on a side stream")
