@@ -73,6 +73,8 @@ def lib() -> ctypes.CDLL:
             L.gemm_k_iterations.argtypes = [I, I]
             L.gemm_tile_coord.argtypes = [ctypes.c_int64, I, I, I, ctypes.POINTER(I),
                                           ctypes.POINTER(I)]
+            L.gemm_splitk_noalloc.argtypes = [I, I, I, P, L64, P, L64, P, L64, P, U, I, I, P]
+            L.gemm_splitk_noalloc.restype = I
             _lib = L
     return _lib
 
@@ -108,6 +110,14 @@ def grouped_gemm(num_groups, group_rows, total_rows, N, K, A, lda, B, ldb, strid
     return lib().grouped_gemm(num_groups, _ptr(group_rows), total_rows, N, K, _ptr(A), lda,
                               _ptr(B), ldb, stride_b, _ptr(C), ldc, _ptr(bias), epilogue, dtype,
                               _stream(stream))
+
+
+def gemm_splitk_noalloc(M, N, K, A, lda, B, ldb, C, ldc, bias, epilogue, dtype, splits,
+                        stream=None) -> int:
+    """C-ABI ``gemm_splitk_noalloc`` (split-K with the library's fixed
+    scratch, no device allocation); returns the gemm_status."""
+    return lib().gemm_splitk_noalloc(M, N, K, _ptr(A), lda, _ptr(B), ldb, _ptr(C), ldc,
+                                     _ptr(bias), epilogue, dtype, splits, _stream(stream))
 
 
 def gemm_status_string(status: int) -> str:

@@ -604,3 +604,138 @@ int gemm_tile_coord(int64_t tile, int grid_m, int grid_n, int group_m, int* m_bl
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Split-K with library-owned scratch (gemm_splitk_noalloc).  The scratch is a
+// fixed array inside this module, so the entry point never allocates.
+
+// One array per device that loads the library: 16 KiB of tile counters, then
+// fp32 partial tiles.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[GEMM_NOALLOC_SCRATCH_BYTES];
+
+namespace dg16 {
+namespace {
+
+constexpr size_t kNoAllocCounterSlots = 4096;
+constexpr size_t kNoAllocCounterBytes = kNoAllocCounterSlots * sizeof(unsigned);
+constexpr int kNoAllocTileConfig = 1;  // tc1_128x128_s6_g8
+constexpr int kNoAllocSwapConfig = 2;  // swap_128x16_s8
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code
+// `g_noalloc_scratch` names a host-side stand-in, not device memory, so its
+// address is looked up once per device (with that device current).
+int noalloc_scratch(void** out) {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kMaxDevices) return GEMM_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return GEMM_OK;
+}
+
+}  // namespace
+}  // namespace dg16
+
+extern "C" int gemm_splitk_noalloc(int M, int N, int K, const void* A, int64_t lda,
+                                   const void* B, int64_t ldb, void* C, int64_t ldc,
+                                   const void* bias, unsigned epilogue, int dtype, int splits,
+                                   void* stream_) {
+  int rc = check_dtype_epi(epilogue, dtype);
+  if (rc) return rc;
+  if (M < 0 || N < 0 || K < 0 || splits < 1 || splits > 64) return GEMM_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return GEMM_OK;
+  rc = check_common(N, K, A, lda, B, ldb, C, ldc, bias, epilogue, dtype);
+  if (rc) return rc;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc) return rc;
+  if (K == 0) return fill_dispatch(M, N, C, ldc, bias, epilogue, dtype, stream);
+
+  const bool bcol = (epilogue & GEMM_B_COL_MAJOR) != 0;
+  const bool bf16 = in_bf16(dtype);
+  const bool f32 = out_bytes(dtype) == 4;
+  const bool swap = bcol && M <= 32;
+  const Config& cfg = kConfigs[swap ? kNoAllocSwapConfig : kNoAllocTileConfig];
+  const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false);
+  if (!k.fn) return GEMM_ERR_UNSUPPORTED;
+
+  KParams kp = {};
+  kp.M = M;
+  kp.N = N;
+  kp.K = K;
+  kp.num_kb = (K + kBK - 1) / kBK;
+  kp.group_m = cfg.group_m;
+  kp.C = C;
+  kp.ldc = ldc;
+  kp.bias = bias;
+  kp.epi = static_cast<int>(epilogue & 3);
+  kp.pol_p = cfg.pol_p;
+  kp.pol_q = cfg.pol_q;
+  kp.num_p = swap ? (N + kBM - 1) / kBM : (M + kBM - 1) / kBM;
+  kp.num_q = swap ? (M + cfg.bn - 1) / cfg.bn : (N + cfg.bn - 1) / cfg.bn;
+  kp.num_tiles = static_cast<long long>(kp.num_p) * kp.num_q;
+  const int per = (kp.num_kb + splits - 1) / splits;
+  kp.kb_per_split = per;
+  kp.splits = (kp.num_kb + per - 1) / per;  // no empty K range
+  const size_t partial = static_cast<size_t>(kp.num_tiles) * kp.splits * kBM * cfg.bn * 4;
+  if (kp.splits > 1 && (kp.num_tiles > static_cast<long long>(kNoAllocCounterSlots) ||
+                        partial > GEMM_NOALLOC_SCRATCH_BYTES - kNoAllocCounterBytes))
+    return GEMM_ERR_UNSUPPORTED;  // beyond the fixed scratch
+  rc = ensure_smem_attr(ds, k);
+  if (rc) return rc;
+
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  kp.counters = static_cast<unsigned*>(scratch);
+  kp.ws = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoAllocCounterBytes);
+  kp.status = ds->status;
+  kp.timeout_ns = g_timeout_ns.load();
+
+  CUtensorMap tp, tq;
+  const uint64_t lda_b = static_cast<uint64_t>(lda) * 2, ldb_b = static_cast<uint64_t>(ldb) * 2;
+  if (!swap) {
+    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
+    rc = make_map(&tp, A, bf16, 2, dA, &lda_b, bA);
+    if (rc) return rc;
+    if (bcol) {
+      const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+      const uint32_t bB[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn)};
+      rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
+    } else {
+      const uint64_t dB[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K)};
+      const uint32_t bB[2] = {64u, static_cast<uint32_t>(kBK)};
+      rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
+    }
+    if (rc) return rc;
+  } else {
+    const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
+    const uint32_t bB[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
+    rc = make_map(&tp, B, bf16, 2, dB, &ldb_b, bB);
+    if (rc) return rc;
+    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
+    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn)};
+    rc = make_map(&tq, A, bf16, 2, dA, &lda_b, bA);
+    if (rc) return rc;
+  }
+  if (kp.splits > 1) {
+    // counters left by an earlier call that gave up early must not leak in
+    cudaError_t e = cudaMemsetAsync(kp.counters, 0,
+                                    static_cast<size_t>(kp.num_tiles) * sizeof(unsigned), stream);
+    if (e != cudaSuccess) return cuda_fail(e);
+  }
+  const int grid =
+      static_cast<int>(std::min<long long>(kp.num_tiles * kp.splits, ds->num_sms));
+  return launch(k, grid, stream, tp, tq, kp);
+}

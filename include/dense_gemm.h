@@ -188,6 +188,46 @@ GEMM_API int gemm_select_config(int M, int N, int K, int dtype, unsigned epilogu
  * GEMM_ERR_UNSUPPORTED.  Returns GEMM_OK or GEMM_ERR_UNSUPPORTED. */
 GEMM_API int gemm_force_config(int id);
 
+/* ---- split-K without any device allocation ------------------------------ */
+
+/* Size of the library's fixed split-K scratch array (bytes per device). */
+#define GEMM_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * gemm_splitk_noalloc -- the split-K GEMM (C = act(A . B + bias), arguments
+ * exactly as for gemm()) with its scratch memory taken from a fixed array that
+ * is part of the library itself, so the call never allocates device memory.
+ * The pages have no counterpart to this entry point.
+ *
+ * Who needs it: gemm() gets its split-K scratch from cudaMalloc, once per
+ * stream.  Some callers cannot allow that -- a service whose device memory
+ * is carved up by its own allocator up front (cudaMalloc behind its back
+ * breaks its accounting or fails once the pool owns the GPU), or a
+ * latency-critical loop that cannot take cudaMalloc's implicit device-wide
+ * synchronisation.  This entry point calls no cudaMalloc, cudaFree or any
+ * other allocating routine.
+ *
+ *   splits   split-K factor, 1..64: each output tile's K range is cut into
+ *            `splits` pieces (fewer if K is short; empty pieces are dropped)
+ *   others   as gemm().  Tiles are 128 x 128, or 128 rows of B by 16 rows
+ *            of A when M <= 32 and B is column-major.
+ * Limits: the scratch holds GEMM_NOALLOC_SCRATCH_BYTES per device: 16 KiB of
+ * tile counters (at most 4096 output tiles) and the fp32 partial tiles
+ * (tiles x pieces x 128 x tile-width x 4 bytes).  A problem that needs more
+ * returns GEMM_ERR_UNSUPPORTED before anything is launched.
+ * Sharing: every call on a device uses the same array, which keeps the last
+ * call's contents; each call first clears the counters it uses on `stream`.
+ * Calls whose kernels overlap on the GPU (different streams, or graph
+ * branches) race on the array and produce wrong results: serialise them.
+ * Set-up: the first call on each device (with that device current) looks up
+ * the array's device address (cudaGetSymbolAddress); make that first call
+ * before any stream capture.  Every GPU that loads the library holds the
+ * array until the process exits.
+ */
+GEMM_API int gemm_splitk_noalloc(int M, int N, int K, const void* A, int64_t lda, const void* B,
+                                 int64_t ldb, void* C, int64_t ldc, const void* bias,
+                                 unsigned epilogue, int dtype, int splits, void* stream);
+
 /* ---- host-side helpers (no GPU needed) --------------------------------- */
 
 /* Bytes of the shared-memory operand ring for a BM x BN output tile with a
