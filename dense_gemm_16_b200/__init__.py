@@ -73,6 +73,9 @@ def lib() -> ctypes.CDLL:
             L.gemm_k_iterations.argtypes = [I, I]
             L.gemm_tile_coord.argtypes = [ctypes.c_int64, I, I, I, ctypes.POINTER(I),
                                           ctypes.POINTER(I)]
+            L.gemm_strided_batched.argtypes = [I, I, I, I, P, L64, L64, P, L64, L64, P, L64, L64,
+                                               P, L64, U, I, P]
+            L.gemm_strided_batched.restype = I
             L.gemm_splitk_noalloc.argtypes = [I, I, I, P, L64, P, L64, P, L64, P, U, I, I, P]
             L.gemm_splitk_noalloc.restype = I
             _lib = L
@@ -102,6 +105,14 @@ def gemm(M, N, K, A, lda, B, ldb, C, ldc, bias, epilogue, dtype, stream=None) ->
     """C-ABI ``gemm``; returns the gemm_status."""
     return lib().gemm(M, N, K, _ptr(A), lda, _ptr(B), ldb, _ptr(C), ldc, _ptr(bias),
                       epilogue, dtype, _stream(stream))
+
+
+def gemm_strided_batched(batch, M, N, K, A, lda, stride_a, B, ldb, stride_b, C, ldc, stride_c,
+                         bias, stride_bias, epilogue, dtype, stream=None) -> int:
+    """C-ABI ``gemm_strided_batched``; returns the gemm_status."""
+    return lib().gemm_strided_batched(batch, M, N, K, _ptr(A), lda, stride_a, _ptr(B), ldb,
+                                      stride_b, _ptr(C), ldc, stride_c, _ptr(bias), stride_bias,
+                                      epilogue, dtype, _stream(stream))
 
 
 def grouped_gemm(num_groups, group_rows, total_rows, N, K, A, lda, B, ldb, stride_b, C, ldc,
@@ -209,6 +220,31 @@ def matmul(a, b, bias=None, relu: bool = False, b_col_major: bool = False, out=N
               stream)
     if rc:
         raise GemmError(rc)
+    return out
+
+
+def bmm(a, b, bias=None, relu: bool = False, b_col_major: bool = False, out=None,
+        out_f32: bool = False, stream=None):
+    """Strided-batched C_i = act(a_i @ B_i + bias_i) through the C ABI.
+
+    a: (batch, M, K); b: (batch, K, N), or (batch, N, K) with
+    ``b_col_major`` (a batch stride of 0 -- e.g. from ``expand`` -- shares
+    one operand across batches); bias: (batch, N) or (N,) or None."""
+    import torch
+    batch, M, K = a.shape
+    N = b.shape[1] if b_col_major else b.shape[2]
+    code = dtype_code(a.dtype, out_f32)
+    if out is None:
+        out = torch.empty(batch, M, N, device=a.device,
+                          dtype=torch.float32 if out_f32 else a.dtype)
+    epi = (GEMM_EPI_BIAS if bias is not None else 0) | (GEMM_EPI_RELU if relu else 0) | \
+        (GEMM_B_COL_MAJOR if b_col_major else 0)
+    sbias = 0 if bias is None or bias.dim() == 1 else bias.stride(0)
+    rc = gemm_strided_batched(batch, M, N, K, a, a.stride(1), a.stride(0), b, b.stride(1),
+                              b.stride(0), out, out.stride(1), out.stride(0), bias, sbias, epi,
+                              code, stream)
+    if rc:
+        raise GemmError(rc, "gemm_strided_batched")
     return out
 
 

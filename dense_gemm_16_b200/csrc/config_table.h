@@ -28,15 +28,19 @@ static const Config kConfigs[] = {
     {"tc1_128x128_s6_g8_k4", kKindSingle, 128, 6, 8, 4, 2, 2},
     {"tc1_128x256_s4_g8_k2", kKindSingle, 256, 4, 8, 2, 2, 2},
     {"pair_256x256_s6_g16", kKindPair, 256, 6, 16, 1, 2, 2},
-    {"pair_256x256_s7_g8", kKindPair, 256, 7, 8, 1, 2, 2},
-    {"pair_256x256_s7_g8_pn", kKindPair, 256, 7, 8, 1, 0, 0},
-    {"pair_256x256_s7_g8_pa", kKindPair, 256, 7, 8, 1, 2, 0},
-    {"pair_256x256_s7_g4", kKindPair, 256, 7, 4, 1, 2, 2},
-    {"tc1_128x256_s4_g8_pn", kKindSingle, 256, 4, 8, 1, 0, 0},
-    {"tc1_128x128_s6_g8_pn", kKindSingle, 128, 6, 8, 1, 0, 0},
     {"pair_256x512_s4_g8", kKindPair, 512, 4, 8, 1, 2, 2},
     {"pair_256x512_s4_g16", kKindPair, 512, 4, 16, 1, 2, 2},
     {"pair_256x512_s4_g8_pn", kKindPair, 512, 4, 8, 1, 0, 0},
+    {"tc1_128x256_s4_g8_pn", kKindSingle, 256, 4, 8, 1, 0, 0},
+    {"tc1_128x128_s6_g8_pn", kKindSingle, 128, 6, 8, 1, 0, 0},
+    {"swap_128x16_s8_k16", kKindSwap, 16, 8, 1, 16, 1, 2},
+    {"swap_128x16_s8_k32", kKindSwap, 16, 8, 1, 32, 1, 2},
+    {"pair_256x512_s4_g16_pf", kKindPair, 512, 4, 16, 1, 2, 1},
+    {"pair_256x512_s4_g32", kKindPair, 512, 4, 32, 1, 2, 2},
+    {"swap_128x16_s8_sk", kKindSwap, 16, 8, 1, -1, 1, 2},
+    {"swap_128x32_s8_sk", kKindSwap, 32, 8, 1, -1, 1, 2},
+    {"tc1_128x128_s6_g8_sk", kKindSingle, 128, 6, 8, -1, 2, 2},
+    {"tc1_128x256_s4_g8_sk", kKindSingle, 256, 4, 8, -1, 2, 2},
 };
 static constexpr int kNumConfigs = static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0]));
 
@@ -55,8 +59,8 @@ static const Rule kRules[] = {
     {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 1},  // m1024n1024k2048: tc1_128x128_s6_g8 215 TFLOP/s
     {2048, 2048, 2048, 2048, 2048, 2048, 0, 0, 0},  // square2048: tc1_128x256_s4_g8 714 TFLOP/s
     {4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 11},  // square4096 (sustained): pair_256x256_s6_g16 1285 TFLOP/s
-    {8192, 8192, 8192, 8192, 8192, 8192, 0, 0, 19},  // square8192 (sustained): pair_256x512_s4_g16 1311 TFLOP/s
-    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 17},  // m1000n1000k2000_bcol: tc1_128x128_s6_g8_pn 186 TFLOP/s
+    {8192, 8192, 8192, 8192, 8192, 8192, 0, 0, 13},  // square8192 (sustained): pair_256x512_s4_g16 1311 TFLOP/s
+    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 16},  // m1000n1000k2000_bcol: tc1_128x128_s6_g8_pn 186 TFLOP/s
     {4096, 4096, 4096, 4096, 512, 512, 1, 0, 1},  // m4096n4096k512_bcol: tc1_128x128_s6_g8 509 TFLOP/s
     {16, 16, 8192, 8192, 8192, 8192, 1, 0, 6},  // m16n8192k8192_bcol: swap_128x16_s8_k4 61 TFLOP/s
     {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 716 TFLOP/s (grouped ignores split-K)
@@ -83,7 +87,7 @@ inline int table_lookup(int M, int N, int K, bool b_col, bool grouped) {
   const long long pair512_tiles = static_cast<long long>((M + 255) / 256) * ((N + 511) / 512);
   // Wide 256 x 512 pair tiles stage the fewest operand bytes per FLOP (the
   // most energy-efficient under the power cap) once there are ~4 waves of them
-  if (!grouped && pair512_tiles >= 296 && K >= 2048) return 19;
+  if (!grouped && pair512_tiles >= 296 && K >= 2048) return 13;
   if (!grouped && pair_tiles >= 128 && K >= 1024) return 11;
   if (N <= 128 || tiles256 < 96) return 1;
   return 0;

@@ -177,10 +177,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return g_encode;
 }
 
-// A 2- or 3-D 16-bit tensor map with 128-byte swizzle and zero fill outside
-// the tensor.  dims[0] is the contiguous dimension; strides in bytes.
-int make_map(CUtensorMap* m, const void* base, bool bf16, int rank, const uint64_t* dims,
-             const uint64_t* strides_bytes, const uint32_t* box) {
+// A 2- or 3-D tensor map with 128-byte swizzle and zero fill outside the
+// tensor.  dims[0] is the contiguous dimension; strides in bytes.
+int make_map_t(CUtensorMap* m, const void* base, CUtensorMapDataType type, int rank,
+               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
   auto enc = encoder();
   if (!enc) return GEMM_ERR_CUDA;
   cuuint64_t gd[3], gs[2];
@@ -190,11 +190,31 @@ int make_map(CUtensorMap* m, const void* base, bool bf16, int rank, const uint64
     bx[i] = box[i];
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-  CUresult r = enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                   rank, const_cast<void*>(base), gd, gs, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, type, rank, const_cast<void*>(base), gd, gs, bx, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_CUDA;
+}
+
+// 16-bit operand map (A or B).
+int make_map(CUtensorMap* m, const void* base, bool bf16, int rank, const uint64_t* dims,
+             const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_map_t(m, base, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                    rank, dims, strides_bytes, box);
+}
+
+// Output map for the TMA-store epilogue: M x N with leading dimension ldc,
+// boxes of 32 rows x 128 bytes (64 16-bit or 32 fp32 outputs).  TMA stores
+// clip at M and N.
+int make_c_map(CUtensorMap* m, void* C, int M, int N, int64_t ldc, int dtype) {
+  const int ob = (dtype == GEMM_F16_OUT_F32 || dtype == GEMM_BF16_OUT_F32) ? 4 : 2;
+  const CUtensorMapDataType t = ob == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                : (dtype == GEMM_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                      : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+  const uint64_t dims[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(M)};
+  const uint64_t stride = static_cast<uint64_t>(ldc) * ob;
+  const uint32_t box[2] = {static_cast<uint32_t>(128 / ob), 32u};
+  return make_map_t(m, C, t, 2, dims, &stride, box);
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -241,7 +261,7 @@ KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool gro
 }
 
 int launch(const KernelEntry& k, int grid, cudaStream_t stream, const CUtensorMap& tp,
-           const CUtensorMap& tq, const KParams& kp, int cluster = 1) {
+           const CUtensorMap& tq, const CUtensorMap& tc, const KParams& kp, int cluster = 1) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(grid, 1, 1);
@@ -258,8 +278,8 @@ int launch(const KernelEntry& k, int grid, cudaStream_t stream, const CUtensorMa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  void* args[3] = {const_cast<CUtensorMap*>(&tp), const_cast<CUtensorMap*>(&tq),
-                   const_cast<KParams*>(&kp)};
+  void* args[4] = {const_cast<CUtensorMap*>(&tp), const_cast<CUtensorMap*>(&tq),
+                   const_cast<CUtensorMap*>(&tc), const_cast<KParams*>(&kp)};
   cudaError_t e = cudaLaunchKernelExC(&cfg, k.fn, args);
   return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
 }
@@ -270,26 +290,222 @@ int select_config(int M, int N, int K, unsigned epi, bool grouped) {
   return table_lookup(M, N, K, (epi & GEMM_B_COL_MAJOR) != 0, grouped);
 }
 
+// One dense (optionally strided-batched) problem as the entry points take it.
+struct DenseProblem {
+  int batch, M, N, K;
+  const void* A;
+  int64_t lda, stride_a;
+  const void* B;
+  int64_t ldb, stride_b;
+  void* C;
+  int64_t ldc, stride_c;
+  const void* bias;
+  int64_t stride_bias;
+  unsigned epi;
+  int dtype;
+};
+
+// Batch strides: an operand is either shared by every batch (stride 0) or
+// its batches do not overlap; outputs never overlap; every stride a TMA map
+// uses is a multiple of 16 bytes.
+int check_batch(const DenseProblem& d) {
+  if (d.stride_a < 0 || d.stride_b < 0 || d.stride_c < 0 || d.stride_bias < 0)
+    return GEMM_ERR_INVALID_ARG;
+  if (d.batch <= 1) return GEMM_OK;
+  const bool bcol = (d.epi & GEMM_B_COL_MAJOR) != 0;
+  const int64_t ext_a = d.lda * d.M;
+  const int64_t ext_b = bcol ? d.ldb * d.N : d.ldb * d.K;
+  if (d.K > 0) {
+    if (d.stride_a != 0 && d.stride_a < ext_a) return GEMM_ERR_INVALID_ARG;
+    if (d.stride_b != 0 && d.stride_b < ext_b) return GEMM_ERR_INVALID_ARG;
+    if ((d.stride_a * 2) % 16 != 0 || (d.stride_b * 2) % 16 != 0) return GEMM_ERR_MISALIGNED;
+  }
+  if (d.stride_c < d.ldc * d.M) return GEMM_ERR_INVALID_ARG;
+  if ((d.stride_c * out_bytes(d.dtype)) % 16 != 0) return GEMM_ERR_MISALIGNED;
+  return GEMM_OK;
+}
+
 template <typename InT, typename OutT>
-int launch_fill(int M, int N, void* C, int64_t ldc, const void* bias, unsigned epi,
-                cudaStream_t stream) {
-  const long long total = static_cast<long long>(M) * N;
+int launch_fill(const DenseProblem& d, cudaStream_t stream) {
+  const long long total = static_cast<long long>(d.M) * d.N * d.batch;
   const int blocks = static_cast<int>(std::min<long long>((total + 255) / 256, 4096));
   fill_bias_kernel<InT, OutT><<<blocks, 256, 0, stream>>>(
-      M, N, static_cast<OutT*>(C), ldc, static_cast<const InT*>(bias), static_cast<int>(epi & 3));
+      d.batch, d.M, d.N, static_cast<OutT*>(d.C), d.ldc, d.batch > 1 ? d.stride_c : 0,
+      static_cast<const InT*>(d.bias), d.batch > 1 ? d.stride_bias : 0,
+      static_cast<int>(d.epi & 3));
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
 }
 
-int fill_dispatch(int M, int N, void* C, int64_t ldc, const void* bias, unsigned epi, int dtype,
-                  cudaStream_t stream) {
-  switch (dtype) {
-    case GEMM_F16: return launch_fill<__half, __half>(M, N, C, ldc, bias, epi, stream);
-    case GEMM_BF16:
-      return launch_fill<__nv_bfloat16, __nv_bfloat16>(M, N, C, ldc, bias, epi, stream);
-    case GEMM_F16_OUT_F32: return launch_fill<__half, float>(M, N, C, ldc, bias, epi, stream);
-    default: return launch_fill<__nv_bfloat16, float>(M, N, C, ldc, bias, epi, stream);
+int fill_dispatch(const DenseProblem& d, cudaStream_t stream) {
+  switch (d.dtype) {
+    case GEMM_F16: return launch_fill<__half, __half>(d, stream);
+    case GEMM_BF16: return launch_fill<__nv_bfloat16, __nv_bfloat16>(d, stream);
+    case GEMM_F16_OUT_F32: return launch_fill<__half, float>(d, stream);
+    default: return launch_fill<__nv_bfloat16, float>(d, stream);
   }
+}
+
+// Fixed scratch for callers that must not allocate (gemm_splitk_noalloc).
+struct FixedScratch {
+  unsigned* counters;
+  size_t counter_slots;
+  float* ws;
+  size_t partial_bytes;
+};
+
+// Plan and launch one dense problem with config `cfg`; `splits` overrides
+// the config's split factor (1 whole tiles, > 1 split-K, -1 stream-K).  The
+// pieces' scratch comes from the per-stream workspace, or from `fixed`.
+int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int splits,
+              const FixedScratch* fixed, cudaStream_t stream) {
+  const int M = d.M, N = d.N, K = d.K;
+  const bool bcol = (d.epi & GEMM_B_COL_MAJOR) != 0;
+  const bool bf16 = in_bf16(d.dtype);
+  const bool f32 = out_bytes(d.dtype) == 4;
+  const bool swap = cfg.kind == kKindSwap;
+  const bool pair = cfg.kind == kKindPair;
+  const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false);
+  if (!k.fn || (swap && !bcol)) return GEMM_ERR_UNSUPPORTED;
+
+  // batch extents of the 3-D maps: a shared operand has one batch
+  const bool bat = d.batch > 1;
+  const uint64_t nb_a = (bat && d.stride_a) ? d.batch : 1, nb_b = (bat && d.stride_b) ? d.batch : 1;
+  const uint64_t sa = (bat && d.stride_a) ? d.stride_a : d.lda * M;
+  const uint64_t sb = (bat && d.stride_b) ? d.stride_b : (bcol ? d.ldb * N : d.ldb * K);
+  const uint64_t str_a[2] = {static_cast<uint64_t>(d.lda) * 2, sa * 2};
+  const uint64_t str_b[2] = {static_cast<uint64_t>(d.ldb) * 2, sb * 2};
+
+  CUtensorMap tp, tq, tc;
+  std::memset(&tc, 0, sizeof(tc));  // swapped tiles store from registers
+  const int ob = out_bytes(d.dtype);
+  const bool tma_store = !swap && (static_cast<int64_t>(N) * ob) % 16 == 0;
+  int rc;
+  if (tma_store) {
+    const CUtensorMapDataType t = ob == 4 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                  : (bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    const uint64_t sc = bat ? d.stride_c : d.ldc * M;
+    const uint64_t dims[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                              static_cast<uint64_t>(d.batch)};
+    const uint64_t str[2] = {static_cast<uint64_t>(d.ldc) * ob, sc * ob};
+    const uint32_t box[3] = {static_cast<uint32_t>(128 / ob), 32u, 1u};
+    rc = make_map_t(&tc, d.C, t, 3, dims, str, box);
+    if (rc) return rc;
+  }
+  KParams kp = {};
+  kp.tma_store = tma_store ? 1 : 0;
+  kp.M = M;
+  kp.N = N;
+  kp.K = K;
+  kp.num_kb = (K + kBK - 1) / kBK;
+  kp.group_m = cfg.group_m;
+  kp.C = d.C;
+  kp.ldc = d.ldc;
+  kp.bias = d.bias;
+  kp.epi = static_cast<int>(d.epi & 3);
+  kp.status = ds->status;
+  kp.timeout_ns = g_timeout_ns.load();
+  kp.stride_c = bat ? d.stride_c : 0;
+  kp.stride_bias = bat ? d.stride_bias : 0;
+  if (!swap) {
+    const uint64_t dA[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M), nb_a};
+    const uint32_t bA[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM), 1u};
+    rc = make_map(&tp, d.A, bf16, 3, dA, str_a, bA);
+    if (rc) return rc;
+    if (bcol) {
+      // the pair kernel's CTAs each load half of the tile's B columns
+      // (pair tiles wider than 256 are several N=256 MMAs, each split in two)
+      const uint64_t dB[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), nb_b};
+      const uint32_t rows_b = pair ? static_cast<uint32_t>(std::min(cfg.bn, 256) / 2)
+                                   : static_cast<uint32_t>(cfg.bn);
+      const uint32_t bB[3] = {static_cast<uint32_t>(kBK), rows_b, 1u};
+      rc = make_map(&tq, d.B, bf16, 3, dB, str_b, bB);
+    } else {
+      const uint64_t dB[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K), nb_b};
+      const uint32_t bB[3] = {64u, static_cast<uint32_t>(kBK), 1u};
+      rc = make_map(&tq, d.B, bf16, 3, dB, str_b, bB);
+    }
+    if (rc) return rc;
+    const int rows_per_tile = pair ? 2 * kBM : kBM;
+    kp.num_p = (M + rows_per_tile - 1) / rows_per_tile;
+    kp.num_q = (N + cfg.bn - 1) / cfg.bn;
+    kp.z_p = nb_a > 1 ? 1 : 0;
+    kp.z_q = nb_b > 1 ? 1 : 0;
+  } else {
+    // P = B stored N x K, Q = A (M x K); the accumulator is C^T
+    const uint64_t dB[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), nb_b};
+    const uint32_t bB[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM), 1u};
+    rc = make_map(&tp, d.B, bf16, 3, dB, str_b, bB);
+    if (rc) return rc;
+    const uint64_t dA[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M), nb_a};
+    const uint32_t bA[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn), 1u};
+    rc = make_map(&tq, d.A, bf16, 3, dA, str_a, bA);
+    if (rc) return rc;
+    kp.num_p = (N + kBM - 1) / kBM;
+    kp.num_q = (M + cfg.bn - 1) / cfg.bn;
+    kp.z_p = nb_b > 1 ? 1 : 0;
+    kp.z_q = nb_a > 1 ? 1 : 0;
+  }
+  kp.tiles_per_batch = static_cast<long long>(kp.num_p) * kp.num_q;
+  kp.num_tiles = kp.tiles_per_batch * d.batch;
+  kp.pol_p = cfg.pol_p;
+  kp.pol_q = cfg.pol_q;
+  kp.work_mode = 0;
+  kp.splits = 1;
+  kp.kb_per_split = kp.num_kb;
+  kp.slot_stride = 1;
+  int grid_units = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms));
+  const size_t counter_cap = fixed ? fixed->counter_slots : kCounterSlots;
+  if (!pair && splits != 1 && kp.num_kb >= 2 &&
+      kp.num_tiles <= static_cast<long long>(counter_cap)) {
+    if (splits > 1) {
+      // split-K: every tile's K range in `splits` equal pieces
+      const int per = (kp.num_kb + splits - 1) / splits;
+      kp.work_mode = 1;
+      kp.kb_per_split = per;
+      kp.splits = (kp.num_kb + per - 1) / per;  // no empty K range
+      kp.slot_stride = kp.splits;
+      grid_units = static_cast<int>(std::min<long long>(kp.num_tiles * kp.splits, ds->num_sms));
+    } else {
+      // stream-K: every block gets an equal share of the (tile, K block)
+      // iterations, cut at tile edges
+      const long long total = kp.num_tiles * kp.num_kb;
+      kp.work_mode = 2;
+      kp.sk_width = (total + ds->num_sms - 1) / ds->num_sms;
+      grid_units = static_cast<int>((total + kp.sk_width - 1) / kp.sk_width);
+      kp.slot_stride = static_cast<int>((kp.num_kb + kp.sk_width - 1) / kp.sk_width) + 1;
+    }
+    if (kp.work_mode == 1 && kp.splits == 1) kp.work_mode = 0;
+  }
+  if (kp.work_mode != 0) {
+    const size_t partial =
+        static_cast<size_t>(kp.num_tiles) * kp.slot_stride * kBM * cfg.bn * 4;
+    if (fixed) {
+      if (partial > fixed->partial_bytes) return GEMM_ERR_UNSUPPORTED;  // beyond the scratch
+      kp.ws = fixed->ws;
+      kp.counters = fixed->counters;
+      // counters left by an earlier call that gave up early must not leak in
+      cudaError_t e = cudaMemsetAsync(kp.counters, 0,
+                                      static_cast<size_t>(kp.num_tiles) * sizeof(unsigned), stream);
+      if (e != cudaSuccess) return cuda_fail(e);
+    } else {
+      int dev = 0;
+      cudaError_t e = cudaGetDevice(&dev);
+      if (e != cudaSuccess) return cuda_fail(e);
+      rc = stream_workspace(dev, stream, partial, &kp.ws, &kp.counters);
+      if (rc) return rc;
+    }
+  } else if (fixed && splits > 1 && kp.num_tiles > static_cast<long long>(counter_cap)) {
+    return GEMM_ERR_UNSUPPORTED;  // beyond the scratch's tile counters
+  }
+  rc = ensure_smem_attr(ds, k);
+  if (rc) return rc;
+  if (pair) {
+    const int pairs = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms / 2));
+    return launch(k, 2 * pairs, stream, tp, tq, tc, kp, 2);
+  }
+  return launch(k, grid_units, stream, tp, tq, tc, kp);
 }
 
 template <typename InT, typename OutT>
@@ -327,104 +543,32 @@ const char* gemm_status_string(int status) {
 
 int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B, int64_t ldb, void* C,
          int64_t ldc, const void* bias, unsigned epilogue, int dtype, void* stream_) {
+  return gemm_strided_batched(1, M, N, K, A, lda, 0, B, ldb, 0, C, ldc, 0, bias, 0, epilogue, dtype,
+                              stream_);
+}
+
+int gemm_strided_batched(int batch, int M, int N, int K, const void* A, int64_t lda,
+                         int64_t stride_a, const void* B, int64_t ldb, int64_t stride_b, void* C,
+                         int64_t ldc, int64_t stride_c, const void* bias, int64_t stride_bias,
+                         unsigned epilogue, int dtype, void* stream_) {
   int rc = check_dtype_epi(epilogue, dtype);
   if (rc) return rc;
-  if (M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
-  if (M == 0 || N == 0) return GEMM_OK;
+  if (batch < 0 || M < 0 || N < 0 || K < 0) return GEMM_ERR_INVALID_ARG;
+  if (batch == 0 || M == 0 || N == 0) return GEMM_OK;
   rc = check_common(N, K, A, lda, B, ldb, C, ldc, bias, epilogue, dtype);
+  if (rc) return rc;
+  DenseProblem d{batch, M, N, K, A, lda, stride_a, B, ldb, stride_b, C, ldc, stride_c, bias,
+                 stride_bias, epilogue, dtype};
+  rc = check_batch(d);
   if (rc) return rc;
   cudaStream_t stream = static_cast<cudaStream_t>(stream_);
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
   if (rc) return rc;
-  if (K == 0) return fill_dispatch(M, N, C, ldc, bias, epilogue, dtype, stream);
-
-  const bool bcol = (epilogue & GEMM_B_COL_MAJOR) != 0;
-  const bool bf16 = in_bf16(dtype);
-  const bool f32 = out_bytes(dtype) == 4;
+  if (K == 0) return fill_dispatch(d, stream);
   const int cid = select_config(M, N, K, epilogue, false);
   if (cid < 0 || cid >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
-  const Config& cfg = kConfigs[cid];
-  const bool swap = cfg.kind == kKindSwap;
-  const bool pair = cfg.kind == kKindPair;
-  const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false);
-  if (!k.fn || (swap && !bcol)) return GEMM_ERR_UNSUPPORTED;
-  rc = ensure_smem_attr(ds, k);
-  if (rc) return rc;
-
-  CUtensorMap tp, tq;
-  const uint64_t lda_b = static_cast<uint64_t>(lda) * 2, ldb_b = static_cast<uint64_t>(ldb) * 2;
-  KParams kp = {};
-  kp.M = M;
-  kp.N = N;
-  kp.K = K;
-  kp.num_kb = (K + kBK - 1) / kBK;
-  kp.group_m = cfg.group_m;
-  kp.C = C;
-  kp.ldc = ldc;
-  kp.bias = bias;
-  kp.epi = static_cast<int>(epilogue & 3);
-  kp.status = ds->status;
-  kp.timeout_ns = g_timeout_ns.load();
-  if (!swap) {
-    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
-    rc = make_map(&tp, A, bf16, 2, dA, &lda_b, bA);
-    if (rc) return rc;
-    if (bcol) {
-      // the pair kernel's CTAs each load half of the tile's B columns
-      const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
-      // (pair tiles wider than 256 are several N=256 MMAs, each split in two)
-      const uint32_t rows_b = pair ? static_cast<uint32_t>(std::min(cfg.bn, 256) / 2)
-                                   : static_cast<uint32_t>(cfg.bn);
-      const uint32_t bB[2] = {static_cast<uint32_t>(kBK), rows_b};
-      rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
-    } else {
-      const uint64_t dB[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K)};
-      const uint32_t bB[2] = {64u, static_cast<uint32_t>(kBK)};
-      rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
-    }
-    if (rc) return rc;
-    const int rows_per_tile = pair ? 2 * kBM : kBM;
-    kp.num_p = (M + rows_per_tile - 1) / rows_per_tile;
-    kp.num_q = (N + cfg.bn - 1) / cfg.bn;
-  } else {
-    // P = B stored N x K, Q = A (M x K); the accumulator is C^T
-    const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
-    const uint32_t bB[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
-    rc = make_map(&tp, B, bf16, 2, dB, &ldb_b, bB);
-    if (rc) return rc;
-    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn)};
-    rc = make_map(&tq, A, bf16, 2, dA, &lda_b, bA);
-    if (rc) return rc;
-    kp.num_p = (N + kBM - 1) / kBM;
-    kp.num_q = (M + cfg.bn - 1) / cfg.bn;
-  }
-  kp.num_tiles = static_cast<long long>(kp.num_p) * kp.num_q;
-  kp.pol_p = cfg.pol_p;
-  kp.pol_q = cfg.pol_q;
-  kp.splits = 1;
-  kp.kb_per_split = kp.num_kb;
-  if (!pair && cfg.splits > 1 && kp.num_kb >= 2 &&
-      kp.num_tiles <= static_cast<long long>(kCounterSlots)) {
-    const int per = (kp.num_kb + cfg.splits - 1) / cfg.splits;
-    kp.kb_per_split = per;
-    kp.splits = (kp.num_kb + per - 1) / per;  // no empty K range
-    const size_t partial = static_cast<size_t>(kp.num_tiles) * kp.splits * kBM * cfg.bn * 4;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return cuda_fail(e);
-    rc = stream_workspace(dev, stream, partial, &kp.ws, &kp.counters);
-    if (rc) return rc;
-  }
-  if (pair) {
-    const int pairs = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms / 2));
-    return launch(k, 2 * pairs, stream, tp, tq, kp, 2);
-  }
-  const int grid =
-      static_cast<int>(std::min<long long>(kp.num_tiles * kp.splits, ds->num_sms));
-  return launch(k, grid, stream, tp, tq, kp);
+  return run_dense(ds, d, kConfigs[cid], kConfigs[cid].splits, nullptr, stream);
 }
 
 int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int N, int K,
@@ -514,13 +658,17 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
   kp.timeout_ns = g_timeout_ns.load();
   kp.pol_p = cfg.pol_p;
   kp.pol_q = cfg.pol_q;
+  kp.work_mode = 0;
   kp.splits = 1;
   kp.kb_per_split = kp.num_kb;
+  kp.slot_stride = 1;
   // upper bound on tiles: each group adds at most one partial row block
   const long long nq = (N + cfg.bn - 1) / cfg.bn;
   const long long max_tiles = (static_cast<long long>(total_rows) / kBM + num_groups) * nq;
+  CUtensorMap tc;
+  std::memset(&tc, 0, sizeof(tc));  // grouped tiles store from registers
   const int grid = static_cast<int>(std::min<long long>(max_tiles, ds->num_sms));
-  return launch(k, grid, stream, tp, tq, kp);
+  return launch(k, grid, stream, tp, tq, tc, kp);
 }
 
 int gemm_device_status(void* stream_, int clear) {
@@ -659,83 +807,17 @@ extern "C" int gemm_splitk_noalloc(int M, int N, int K, const void* A, int64_t l
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
   if (rc) return rc;
-  if (K == 0) return fill_dispatch(M, N, C, ldc, bias, epilogue, dtype, stream);
-
-  const bool bcol = (epilogue & GEMM_B_COL_MAJOR) != 0;
-  const bool bf16 = in_bf16(dtype);
-  const bool f32 = out_bytes(dtype) == 4;
-  const bool swap = bcol && M <= 32;
-  const Config& cfg = kConfigs[swap ? kNoAllocSwapConfig : kNoAllocTileConfig];
-  const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false);
-  if (!k.fn) return GEMM_ERR_UNSUPPORTED;
-
-  KParams kp = {};
-  kp.M = M;
-  kp.N = N;
-  kp.K = K;
-  kp.num_kb = (K + kBK - 1) / kBK;
-  kp.group_m = cfg.group_m;
-  kp.C = C;
-  kp.ldc = ldc;
-  kp.bias = bias;
-  kp.epi = static_cast<int>(epilogue & 3);
-  kp.pol_p = cfg.pol_p;
-  kp.pol_q = cfg.pol_q;
-  kp.num_p = swap ? (N + kBM - 1) / kBM : (M + kBM - 1) / kBM;
-  kp.num_q = swap ? (M + cfg.bn - 1) / cfg.bn : (N + cfg.bn - 1) / cfg.bn;
-  kp.num_tiles = static_cast<long long>(kp.num_p) * kp.num_q;
-  const int per = (kp.num_kb + splits - 1) / splits;
-  kp.kb_per_split = per;
-  kp.splits = (kp.num_kb + per - 1) / per;  // no empty K range
-  const size_t partial = static_cast<size_t>(kp.num_tiles) * kp.splits * kBM * cfg.bn * 4;
-  if (kp.splits > 1 && (kp.num_tiles > static_cast<long long>(kNoAllocCounterSlots) ||
-                        partial > GEMM_NOALLOC_SCRATCH_BYTES - kNoAllocCounterBytes))
-    return GEMM_ERR_UNSUPPORTED;  // beyond the fixed scratch
-  rc = ensure_smem_attr(ds, k);
-  if (rc) return rc;
-
+  const DenseProblem d{1, M, N, K, A, lda, 0, B, ldb, 0, C, ldc, 0, bias, 0, epilogue, dtype};
+  if (K == 0) return fill_dispatch(d, stream);
+  const bool swap = (epilogue & GEMM_B_COL_MAJOR) != 0 && M <= 32;
   void* scratch = nullptr;
   rc = noalloc_scratch(&scratch);
   if (rc) return rc;
-  kp.counters = static_cast<unsigned*>(scratch);
-  kp.ws = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoAllocCounterBytes);
-  kp.status = ds->status;
-  kp.timeout_ns = g_timeout_ns.load();
-
-  CUtensorMap tp, tq;
-  const uint64_t lda_b = static_cast<uint64_t>(lda) * 2, ldb_b = static_cast<uint64_t>(ldb) * 2;
-  if (!swap) {
-    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
-    rc = make_map(&tp, A, bf16, 2, dA, &lda_b, bA);
-    if (rc) return rc;
-    if (bcol) {
-      const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
-      const uint32_t bB[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn)};
-      rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
-    } else {
-      const uint64_t dB[2] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K)};
-      const uint32_t bB[2] = {64u, static_cast<uint32_t>(kBK)};
-      rc = make_map(&tq, B, bf16, 2, dB, &ldb_b, bB);
-    }
-    if (rc) return rc;
-  } else {
-    const uint64_t dB[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N)};
-    const uint32_t bB[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
-    rc = make_map(&tp, B, bf16, 2, dB, &ldb_b, bB);
-    if (rc) return rc;
-    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M)};
-    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn)};
-    rc = make_map(&tq, A, bf16, 2, dA, &lda_b, bA);
-    if (rc) return rc;
-  }
-  if (kp.splits > 1) {
-    // counters left by an earlier call that gave up early must not leak in
-    cudaError_t e = cudaMemsetAsync(kp.counters, 0,
-                                    static_cast<size_t>(kp.num_tiles) * sizeof(unsigned), stream);
-    if (e != cudaSuccess) return cuda_fail(e);
-  }
-  const int grid =
-      static_cast<int>(std::min<long long>(kp.num_tiles * kp.splits, ds->num_sms));
-  return launch(k, grid, stream, tp, tq, kp);
+  FixedScratch fs;
+  fs.counters = static_cast<unsigned*>(scratch);
+  fs.counter_slots = kNoAllocCounterSlots;
+  fs.ws = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoAllocCounterBytes);
+  fs.partial_bytes = GEMM_NOALLOC_SCRATCH_BYTES - kNoAllocCounterBytes;
+  return run_dense(ds, d, kConfigs[swap ? kNoAllocSwapConfig : kNoAllocTileConfig], splits, &fs,
+                   stream);
 }

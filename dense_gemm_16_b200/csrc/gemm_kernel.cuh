@@ -44,7 +44,7 @@ namespace dg16 {
 template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT, bool SWAP, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                   const KParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const KParams p) {
   using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
   static_assert(!Q_MN || BN % 64 == 0, "MN-major Q tiles are whole 64-element swizzle rows");
@@ -52,9 +52,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t P_BYTES = kBM * kBK * 2;
   constexpr uint32_t Q_BYTES = BN * kBK * 2;
   constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
-  constexpr uint32_t TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                 : (2 * BN <= 256) ? 256 : 512;
+  // Swapped (skinny) tiles have a tiny MMA-N, so one accumulator would chain
+  // every MMA of a tile through its latency: consecutive K blocks rotate over
+  // NACC independent accumulators instead, summed in order by the epilogue.
+  constexpr int NACC = SWAP ? (BN <= 16 ? 4 : 2) : 1;
+  constexpr int ACC_COLS = NACC * BN;  // TMEM columns per accumulator buffer
+  constexpr uint32_t TMEM_COLS = (2 * ACC_COLS <= 32) ? 32 : (2 * ACC_COLS <= 64) ? 64
+                                 : (2 * ACC_COLS <= 128) ? 128 : (2 * ACC_COLS <= 256) ? 256 : 512;
   constexpr uint32_t IDESC = f16_idesc(kBM, BN, IN_BF16 ? 1u : 0u, 0u, Q_MN ? 1u : 0u);
+  // dense tiles store through shared memory and TMA; grouped tiles must not
+  // write past their group's last row and swapped tiles are transposed, so
+  // those store from registers
+  constexpr bool TMA_EPI = !GROUPED && !SWAP;
+  constexpr uint32_t STAGE_EPI = TMA_EPI ? kEpiStageBytes : 0u;
 
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128-byte swizzle atoms (8 rows x 128 B)
@@ -62,7 +72,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sP = smem;
   uint8_t* sQ = smem + STAGES * P_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sQ + STAGES * Q_BYTES);
+  uint8_t* sStage = sQ + STAGES * Q_BYTES;  // 1024-aligned epilogue staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + STAGE_EPI);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* accf_bar = bars + 2 * STAGES;
@@ -91,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmP);
     tma_prefetch_desc(&tmQ);
+    if constexpr (TMA_EPI) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc<1>(smem_u32(&ctl->tmem_base), TMEM_COLS);
@@ -129,10 +141,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   long long num_tiles = p.num_tiles;
   if constexpr (GROUPED) num_tiles = gt->tile_start[p.num_groups];
   const int num_q_blocks = GROUPED ? (p.N + BN - 1) / BN : p.num_q;
-  // Work units: (tile, K range).  Without split-K a unit is a whole tile.
-  const int splits = GROUPED ? 1 : p.splits;
-  const int kb_per = splits > 1 ? p.kb_per_split : p.num_kb;
-  const long long num_units = num_tiles * splits;
 
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer
@@ -142,14 +150,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       int gcur = 0;
       bool ok = true;
-      for (long long u = blockIdx.x; u < num_units && ok; u += gridDim.x) {
-        const long long t = u / splits;
-        const int kb0 = static_cast<int>(u % splits) * kb_per;
-        const int kb1 = min(kb0 + kb_per, p.num_kb);
-        const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
+      WorkIter wi(p, num_tiles);
+      Work w;
+      while (ok && wi.next(p, w)) {
+        const TileCoord c = tile_coord<GROUPED>(w.t, p, num_q_blocks, gt, gcur);
         if (!c.valid) break;
         const int q0 = c.q0 * BN;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_phase(smem_u32(&empty_bar[s]), ph ^ 1u, ctl, p, kStatusTimeoutProducer)) {
@@ -158,25 +165,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t fb = smem_u32(&full_bar[s]);
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
-          tma_load_2d(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, c.p0, fb, pol_p);
+          if constexpr (GROUPED)
+            tma_load_2d(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, c.p0, fb, pol_p);
+          else
+            tma_load_3d(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, c.p0, c.zp, fb, pol_p);
           const uint32_t qdst = smem_u32(sQ + s * Q_BYTES);
-          if constexpr (GROUPED) {
-            if constexpr (Q_MN) {
+          // Q is 3-D: [group][rows][cols] (grouped) or [batch][rows][cols]
+          if constexpr (Q_MN) {
 #pragma unroll
-              for (int j = 0; j < BN / 64; ++j)
-                tma_load_3d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, c.group, fb,
-                            pol_q);
-            } else {
-              tma_load_3d(qdst, &tmQ, kb * kBK, q0, c.group, fb, pol_q);
-            }
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_3d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, c.zq, fb,
+                          pol_q);
           } else {
-            if constexpr (Q_MN) {
-#pragma unroll
-              for (int j = 0; j < BN / 64; ++j)
-                tma_load_2d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, fb, pol_q);
-            } else {
-              tma_load_2d(qdst, &tmQ, kb * kBK, q0, fb, pol_q);
-            }
+            tma_load_3d(qdst, &tmQ, kb * kBK, q0, c.zq, fb, pol_q);
           }
         }
       }
@@ -194,18 +195,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, local = 0;
       int gcur = 0;
       bool ok = true;
-      for (long long u = blockIdx.x; u < num_units && ok; u += gridDim.x, ++local) {
-        const long long t = u / splits;
-        const int kb0 = static_cast<int>(u % splits) * kb_per;
-        const int kb1 = min(kb0 + kb_per, p.num_kb);
-        const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
+      WorkIter wi(p, num_tiles);
+      Work w;
+      for (; ok && wi.next(p, w); ++local) {
+        const TileCoord c = tile_coord<GROUPED>(w.t, p, num_q_blocks, gt, gcur);
         if (!c.valid) break;
         const uint32_t a = local & 1u;
         const uint32_t aph = (local >> 1) & 1u;
         if (!wait_phase(smem_u32(&acce_bar[a]), aph ^ 1u, ctl, p, kStatusTimeoutMma)) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + a * BN;
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const uint32_t d0 = tmem_base + a * ACC_COLS;
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
+          const int r = (kb - w.kb0) % NACC;            // accumulator of this K block
+          const uint32_t d = d0 + static_cast<uint32_t>(r * BN);
+          const bool fresh = kb - w.kb0 < NACC;         // its first K block
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_phase(smem_u32(&full_bar[s]), ph, ctl, p, kStatusTimeoutMma)) {
@@ -224,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // kBK rows apart; 8-row K groups 1024 B apart.
             const uint64_t bdesc = Q_MN ? sw128_desc(qbase + k * 16 * 128, kBK * 128, 1024)
                                         : sw128_desc(qbase + k * 32, 16, 1024);
-            mma_f16<1>(d, adesc, bdesc, IDESC, (kb != kb0 || k != 0) ? 1u : 0u);
+            mma_f16<1>(d, adesc, bdesc, IDESC, (!fresh || k != 0) ? 1u : 0u);
           }
           mma_commit<1>(smem_u32(&empty_bar[s]));  // frees the stage when read
         }
@@ -240,24 +243,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ----------------------------------------------------------- epilogue
     const int quad = warp & 3;  // TMEM lanes this warp may read: 32*quad ..
     const int row_local = quad * 32 + lane;
+    const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>(warp - 2) * 8192u;
+    uint32_t stores = 0;  // this warp's TMA stores so far
     uint32_t local = 0;
     int gcur = 0;
-    OutT* C = reinterpret_cast<OutT*>(p.C);
-    const InT* bias = reinterpret_cast<const InT*>(p.bias);
+    OutT* const C0 = reinterpret_cast<OutT*>(p.C);
+    const InT* const bias = reinterpret_cast<const InT*>(p.bias);
     const bool has_bias = (p.epi & 1) != 0;
     const bool relu = (p.epi & 2) != 0;
-    for (long long u = blockIdx.x; u < num_units; u += gridDim.x, ++local) {
-      const long long t = u / splits;
-      const int split = static_cast<int>(u % splits);
-      const TileCoord c = tile_coord<GROUPED>(t, p, num_q_blocks, gt, gcur);
+    const bool pieces_possible = p.work_mode != 0;  // uniform for the launch
+    constexpr long long PART = static_cast<long long>(kBM) * BN;  // floats per partial tile
+    WorkIter wi(p, num_tiles);
+    Work w;
+    for (; wi.next(p, w); ++local) {
+      const TileCoord c = tile_coord<GROUPED>(w.t, p, num_q_blocks, gt, gcur);
       if (!c.valid) break;
       const uint32_t a = local & 1u;
       const uint32_t aph = (local >> 1) & 1u;
       // every lane waits; the warp proceeds only if all saw the phase, so the
       // .sync.aligned TMEM loads below are always issued by the whole warp
       const bool ok = wait_phase(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
-      if (splits > 1) {
-        // the split-K path below syncs the four epilogue warps, so they must
+      if (pieces_possible) {
+        // the piece path below syncs the four epilogue warps, so they must
         // agree on leaving: a failed wait always raises the abort flag first
         epilogue_bar();
         if (*reinterpret_cast<volatile int*>(&ctl->abort)) break;
@@ -267,95 +274,96 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const int prow = c.p0 + row_local;  // this thread's accumulator row
       const int q0 = c.q0 * BN;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * BN;
-      if (splits > 1) {
-        // ---- split-K: park this K range's partial tile, the last range sums
-        float* part = p.ws + (t * splits + split) * static_cast<long long>(kBM * BN) +
-                      static_cast<long long>(row_local) * BN;
+      // this tile's output and bias (grouped: the group's bias row; dense:
+      // the batch's output and bias)
+      OutT* const C = GROUPED ? C0 : C0 + static_cast<long long>(c.group) * p.stride_c;
+      const InT* const bias_t =
+          !has_bias ? nullptr
+                    : (GROUPED ? bias + static_cast<long long>(c.group) * p.N
+                               : bias + static_cast<long long>(c.group) * p.stride_bias);
+      const uint32_t taddr =
+          tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * ACC_COLS;
+      const TmemSrc tsrc{taddr, min(NACC, w.kb1 - w.kb0), BN};
+      bool finish = true;  // this block stores the tile
+      const float* tile0 = nullptr;
+      if (w.count > 1) {
+        // ---- one piece of a split tile: park the partial, the last piece sums
+        float* part = p.ws + (w.t * p.slot_stride + w.idx) * PART;
 #pragma unroll 1
         for (int cc = 0; cc < BN; cc += 16) {
           uint32_t v[16];
-          tmem_ld_32x32b_x16(taddr + cc, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            __stcg(reinterpret_cast<float4*>(part + cc) + j,
-                   make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+          tsrc.get<16>(cc, v);
+          put_partial16(part, row_local, cc, v);
         }
         tc_fence_before();
         mbar_arrive(smem_u32(&acce_bar[a]));  // the accumulator is free again
         __threadfence();
         epilogue_bar();
         if (row_local == 0) {
-          const unsigned old = atomicAdd(&p.counters[t], 1u);
-          ctl->last = (old == static_cast<unsigned>(splits - 1)) ? 1 : 0;
+          const unsigned old = atomicAdd(&p.counters[w.t], 1u);
+          ctl->last = (old == static_cast<unsigned>(w.count - 1)) ? 1 : 0;
         }
         epilogue_bar();
-        if (ctl->last) {
+        finish = ctl->last != 0;
+        if (finish) {
           __threadfence();
-          const float* base = p.ws + t * splits * static_cast<long long>(kBM * BN) +
-                              static_cast<long long>(row_local) * BN;
-          if constexpr (!SWAP) {
-            const InT* bias_g = has_bias ? bias : nullptr;
-            store_partial_sums<BN, InT, OutT>(base, splits, prow, c.row_end, q0, p, bias_g,
-                                              relu, C);
+          tile0 = p.ws + w.t * p.slot_stride * PART;
+        }
+      }
+      if (finish) {
+        const PartialSrc psrc{tile0, PART, w.count, row_local};
+        if constexpr (!SWAP) {
+          const InT* bias_g = bias_t;
+          if (TMA_EPI && p.tma_store) {
+            if (w.count > 1)
+              store_tma_from<BN, InT, OutT>(psrc, c.p0 + quad * 32, q0, c.group, p, bias_g, relu,
+                                            stage, stores, &tmC);
+            else
+              store_tma_from<BN, InT, OutT>(tsrc, c.p0 + quad * 32, q0, c.group, p, bias_g, relu,
+                                            stage, stores, &tmC);
           } else {
-            const bool col_ok = prow < p.N;
-            const float b = (has_bias && col_ok) ? to_f32<InT>(bias[prow]) : 0.0f;
+            // accumulator row = output row prow, columns q0 .. q0+BN
+            if (w.count > 1)
+              store_rows_from<BN, InT, OutT>(psrc, prow, c.row_end, q0, p, bias_g, relu, C);
+            else
+              store_rows_from<BN, InT, OutT>(tsrc, prow, c.row_end, q0, p, bias_g, relu, C);
+          }
+        } else {
+          // accumulator row = output column prow (an N index); accumulator
+          // columns are output rows q0 .. q0+BN
+          const bool col_ok = prow < p.N;
+          const float b = (has_bias && col_ok) ? to_f32<InT>(bias_t[prow]) : 0.0f;
 #pragma unroll 1
-            for (int cc = 0; cc < BN; cc += 16) {
-              const int row0 = q0 + cc;
-              if (row0 >= p.M) break;
-              float f[16];
-              sum_partials16(base + cc, splits, static_cast<long long>(kBM * BN), f);
-              if (col_ok) {
+          for (int cc = 0; cc < BN; cc += 16) {
+            const int row0 = q0 + cc;
+            if (row0 >= p.M) break;  // warp-uniform
+            uint32_t v[16];
+            if (w.count > 1)
+              psrc.get<16>(cc, v);
+            else
+              tsrc.get<16>(cc, v);
+            if (col_ok) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  if (row0 + j < p.M) {
-                    float x = f[j] + b;
-                    if (relu) x = fmaxf(x, 0.0f);
-                    C[static_cast<long long>(row0 + j) * p.ldc + prow] = from_f32<OutT>(x);
-                  }
+              for (int j = 0; j < 16; ++j) {
+                if (row0 + j < p.M) {
+                  float x = __uint_as_float(v[j]) + b;
+                  if (relu) x = fmaxf(x, 0.0f);
+                  C[static_cast<long long>(row0 + j) * p.ldc + prow] = from_f32<OutT>(x);
                 }
               }
             }
           }
-          if (row_local == 0) p.counters[t] = 0u;  // ready for the next launch
         }
-        continue;
+        if (w.count > 1 && row_local == 0) p.counters[w.t] = 0u;  // ready for the next launch
       }
-      if constexpr (!SWAP) {
-        // accumulator row = output row prow, columns q0 .. q0+BN
-        const InT* bias_g = has_bias ? bias + static_cast<long long>(c.group) * p.N : nullptr;
-        store_acc_rows<BN, InT, OutT>(taddr, prow, c.row_end, q0, p, bias_g, relu, C);
-      } else {
-        // accumulator row = output column prow (an N index); accumulator
-        // columns are output rows q0 .. q0+BN
-        const bool col_ok = prow < p.N;
-        const float b = (has_bias && col_ok) ? to_f32<InT>(bias[prow]) : 0.0f;
-#pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 16) {
-          const int row0 = q0 + cc;
-          if (row0 >= p.M) break;  // warp-uniform
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(taddr + cc, v);
-          tmem_ld_wait();
-          if (col_ok) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (row0 + j < p.M) {
-                float x = __uint_as_float(v[j]) + b;
-                if (relu) x = fmaxf(x, 0.0f);
-                C[static_cast<long long>(row0 + j) * p.ldc + prow] = from_f32<OutT>(x);
-              }
-            }
-          }
-        }
+      if (w.count == 1) {
+        tc_fence_before();
+        mbar_arrive(smem_u32(&acce_bar[a]));
       }
-      tc_fence_before();
-      mbar_arrive(smem_u32(&acce_bar[a]));
     }
+    // every TMA store has finished with shared memory (and the output is
+    // written) before the block retires
+    if (TMA_EPI && lane == 0) tma_store_wait_all<0>();
   }
 
   tc_fence_before();
@@ -368,22 +376,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Shared memory a kernel instance needs (bytes, including alignment slack).
-template <int BN, int STAGES, bool GROUPED>
+template <int BN, int STAGES, bool GROUPED, bool SWAP = false>
 constexpr int gemm_smem_bytes() {
-  return 1024 + STAGES * (kBM * kBK * 2 + BN * kBK * 2) + (2 * STAGES + 5) * 8 +
+  return 1024 + STAGES * (kBM * kBK * 2 + BN * kBK * 2) +
+         ((!GROUPED && !SWAP) ? static_cast<int>(kEpiStageBytes) : 0) + (2 * STAGES + 5) * 8 +
          static_cast<int>(sizeof(SharedCtl)) + (GROUPED ? static_cast<int>(sizeof(GroupTable)) : 0);
 }
 
-// C = act(bias) (or zeros) for K == 0: the definition with an empty sum.
+// C = act(bias) (or zeros) for K == 0: the definition with an empty sum,
+// for `batch` outputs stride_c elements apart (bias stride_bias apart).
 template <typename InT, typename OutT>
-__global__ void fill_bias_kernel(int M, int N, OutT* C, long long ldc, const InT* bias, int epi) {
-  const long long total = static_cast<long long>(M) * N;
+__global__ void fill_bias_kernel(int batch, int M, int N, OutT* C, long long ldc,
+                                 long long stride_c, const InT* bias, long long stride_bias,
+                                 int epi) {
+  const long long per = static_cast<long long>(M) * N;
+  const long long total = per * batch;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int r = static_cast<int>(i / N), c = static_cast<int>(i % N);
-    float x = (epi & 1) ? to_f32<InT>(bias[c]) : 0.0f;
+    const long long b = i / per, rc = i - b * per;
+    const int r = static_cast<int>(rc / N), c = static_cast<int>(rc % N);
+    float x = (epi & 1) ? to_f32<InT>(bias[b * stride_bias + c]) : 0.0f;
     if (epi & 2) x = fmaxf(x, 0.0f);
-    C[static_cast<long long>(r) * ldc + c] = from_f32<OutT>(x);
+    C[b * stride_c + static_cast<long long>(r) * ldc + c] = from_f32<OutT>(x);
   }
 }
 

@@ -34,7 +34,7 @@ namespace dg16 {
 template <int BN, int NSUB, int STAGES, bool Q_MN, bool IN_BF16, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                    const KParams p) {
+                    const __grid_constant__ CUtensorMap tmC, const KParams p) {
   using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
   constexpr int HALF_N = BN / 2;
   constexpr int TILE_N = BN * NSUB;                 // output columns per pair tile
@@ -54,7 +54,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (raw_addr & 1023u)) & 1023u);
   uint8_t* sP = smem;
   uint8_t* sQ = smem + STAGES * P_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sQ + STAGES * Q_BYTES);
+  uint8_t* sStage = sQ + STAGES * Q_BYTES;  // 1024-aligned epilogue staging
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + kEpiStageBytes);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* accf_bar = bars + 2 * STAGES;
@@ -88,6 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmP);
     tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc<2>(smem_u32(&ctl->tmem_base), TMEM_COLS);
@@ -108,8 +110,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (long long t = pair_id; t < num_tiles && ok; t += num_pairs) {
+        const long long b = t / p.tiles_per_batch;
         int pb, qb;
-        raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
+        raster_tile(t - b * p.tiles_per_batch, p.num_p, p.num_q, p.group_m, pb, qb);
+        const int zp = static_cast<int>(b) * p.z_p, zq = static_cast<int>(b) * p.z_q;
         const int prow0 = pb * (2 * kBM) + static_cast<int>(rank) * kBM;
         // MMA j of the K step covers tile columns [j*BN, (j+1)*BN); this CTA
         // supplies the rank-th half of each
@@ -124,7 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // the leader's full barrier counts both CTAs' bytes
           const uint32_t fb_leader = map_shared_rank(smem_u32(&full_bar[s]), 0);
           if (rank == 0) mbar_arrive_expect_tx(smem_u32(&full_bar[s]), 2 * STAGE_BYTES);
-          tma_load_2d_pair(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, prow0, fb_leader, pol_p);
+          tma_load_3d_pair(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, prow0, zp, fb_leader,
+                           pol_p);
 #pragma unroll
           for (int sub = 0; sub < NSUB; ++sub) {
             const uint32_t qdst = smem_u32(sQ + s * Q_BYTES + sub * QSUB_BYTES);
@@ -132,10 +137,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if constexpr (Q_MN) {
 #pragma unroll
               for (int j = 0; j < HALF_N / 64; ++j)
-                tma_load_2d_pair(qdst + j * (64 * kBK * 2), &tmQ, qc + 64 * j, kb * kBK,
+                tma_load_3d_pair(qdst + j * (64 * kBK * 2), &tmQ, qc + 64 * j, kb * kBK, zq,
                                  fb_leader, pol_q);
             } else {
-              tma_load_2d_pair(qdst, &tmQ, kb * kBK, qc, fb_leader, pol_q);
+              tma_load_3d_pair(qdst, &tmQ, kb * kBK, qc, zq, fb_leader, pol_q);
             }
           }
         }
@@ -203,26 +208,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // --------------------------------------------- epilogue (both CTAs)
     const int quad = warp & 3;
+    const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>(warp - 2) * 8192u;
+    uint32_t stores = 0;
     uint32_t local = 0;
-    OutT* C = reinterpret_cast<OutT*>(p.C);
     const InT* bias = (p.epi & 1) ? reinterpret_cast<const InT*>(p.bias) : nullptr;
     const bool relu = (p.epi & 2) != 0;
     const uint32_t acce_leader0 = map_shared_rank(smem_u32(&acce_bar[0]), 0);
     for (long long t = pair_id; t < num_tiles; t += num_pairs, ++local) {
+      const long long b = t / p.tiles_per_batch;
       int pb, qb;
-      raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
+      raster_tile(t - b * p.tiles_per_batch, p.num_p, p.num_q, p.group_m, pb, qb);
+      const InT* const bias_t = bias ? bias + b * p.stride_bias : nullptr;
       const uint32_t a = ACC_BUFS == 2 ? (local & 1u) : 0u;
       const uint32_t aph = ACC_BUFS == 2 ? ((local >> 1) & 1u) : (local & 1u);
       const bool ok = wait_phase<true>(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int prow = pb * (2 * kBM) + static_cast<int>(rank) * kBM + quad * 32 + lane;
+      const int row0 = pb * (2 * kBM) + static_cast<int>(rank) * kBM + quad * 32;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * TILE_N;
-      store_acc_rows<TILE_N, InT, OutT>(taddr, prow, p.M, qb * TILE_N, p, bias, relu, C);
+      const TmemSrc tsrc{taddr};
+      if (p.tma_store)
+        store_tma_from<TILE_N, InT, OutT>(tsrc, row0, qb * TILE_N, static_cast<int>(b), p, bias_t,
+                                          relu, stage, stores, &tmC);
+      else
+        store_rows_from<TILE_N, InT, OutT>(tsrc, row0 + lane, p.M, qb * TILE_N, p, bias_t, relu,
+                                           reinterpret_cast<OutT*>(p.C) + b * p.stride_c);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader0 + a * 8u);
     }
+    if (lane == 0) tma_store_wait_all<0>();
   }
 
   tc_fence_before();
@@ -237,8 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 template <int BN, int NSUB, int STAGES>
 constexpr int gemm_pair_smem_bytes() {
-  return 1024 + STAGES * (kBM * kBK * 2 + NSUB * (BN / 2) * kBK * 2) + (2 * STAGES + 5) * 8 +
-         static_cast<int>(sizeof(SharedCtl));
+  return 1024 + STAGES * (kBM * kBK * 2 + NSUB * (BN / 2) * kBK * 2) +
+         static_cast<int>(kEpiStageBytes) + (2 * STAGES + 5) * 8 + static_cast<int>(sizeof(SharedCtl));
 }
 
 }  // namespace dg16

@@ -1,8 +1,8 @@
 // Kernel instances of the CTA-pair GEMM: 256 x 512 pair tiles (two N=256
 // MMAs per K step, one 512-column accumulator) with a 4-deep ring of 48 KB
-// stages; 256 x 256 pair tiles with a 6- or 7-deep ring (32 KB per stage per
-// CTA; 7 stages fill 224 KB of the 227 KB a block may use); 256 x 128 pair
-// tiles with an 8-deep ring.
+// stages; 256 x 256 pair tiles with a 6-deep ring (32 KB per stage per CTA);
+// 256 x 128 pair tiles with an 8-deep ring.  Each ring plus the 32 KB
+// epilogue staging area fits the 227 KB a block may use.
 #include "dispatch.h"
 #include "gemm_kernel_pair.cuh"
 
@@ -34,7 +34,6 @@ static KernelEntry pick(bool q_mn, bool bf16, bool f32) {
 // bn = output columns per pair tile (256 x bn)
 KernelEntry kernels_pair(int bn, int stages, bool q_mn, bool bf16, bool out_f32) {
   if (bn == 512) return pick<256, 2, 4>(q_mn, bf16, out_f32);
-  if (bn == 256 && stages == 7) return pick<256, 1, 7>(q_mn, bf16, out_f32);
   if (bn == 256) return pick<256, 1, 6>(q_mn, bf16, out_f32);
   if (bn == 128) return pick<128, 1, 8>(q_mn, bf16, out_f32);
   return {nullptr, 0};

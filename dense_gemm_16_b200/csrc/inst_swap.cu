@@ -12,7 +12,7 @@ static KernelEntry entry_swap() {
   using Out = typename std::conditional<F32, float, In>::type;
   constexpr int S = 8;
   return {reinterpret_cast<const void*>(&gemm_tc_kernel<BN, S, false, BF16, Out, true, false>),
-          gemm_smem_bytes<BN, S, false>()};
+          gemm_smem_bytes<BN, S, false, true>()};
 }
 
 KernelEntry kernels_swap(int bn, bool bf16, bool out_f32) {

@@ -44,12 +44,32 @@ struct KParams {
   unsigned* status;       // device status word
   unsigned long long timeout_ns;
   int pol_p, pol_q;       // L2 policy of the P / Q operand copies (kPolicy*)
-  // split-K: each tile's K blocks are cut into `splits` ranges of kb_per_split
-  // blocks; partial fp32 tiles go to `ws` and the last range to finish sums
-  // them (in range order) and runs the epilogue.  splits == 1: no split.
+  // Work distribution (see WorkIter):
+  //   work_mode 0  whole tiles
+  //   work_mode 1  split-K: each tile's K blocks in `splits` ranges of
+  //                kb_per_split blocks
+  //   work_mode 2  stream-K: block b takes iterations [b*sk_width,
+  //                (b+1)*sk_width) of the (tile, K block) space
+  // A tile computed in several pieces parks fp32 partial tiles in `ws`
+  // (slot tile*slot_stride + piece) and the last piece to finish sums them
+  // in piece order and runs the epilogue.
+  int work_mode;
   int splits, kb_per_split;
-  float* ws;              // [tile][split][128][BN] fp32 partials
+  long long sk_width;
+  int slot_stride;
+  float* ws;              // [slot][BN/4][128][4] fp32 partials
   unsigned* counters;     // [tile] arrivals, left at 0 after every launch
+  // 1: store output tiles with TMA (set only when a row of C ends on a
+  // 16-byte boundary, N * sizeof(out) % 16 == 0: a TMA store writes whole
+  // 16-byte granules, so a shorter row end would spill into the padding)
+  int tma_store;
+  // Strided batches (dense kernels): tile t belongs to batch t / tiles_per_batch.
+  // The operand maps are 3-D with the batch as the third coordinate; an
+  // operand shared by all batches (stride 0) has z_p or z_q == 0.
+  long long tiles_per_batch;
+  int z_p, z_q;           // 1: the P / Q operand advances with the batch
+  long long stride_c;     // elements between batches' outputs
+  long long stride_bias;  // elements between batches' bias vectors
 };
 
 enum : int { kPolicyNormal = 0, kPolicyFirst = 1, kPolicyLast = 2 };
@@ -63,6 +83,62 @@ __device__ __forceinline__ uint64_t make_policy(int code) {
 __device__ __forceinline__ void epilogue_bar() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
+
+// One unit of work: K blocks [kb0, kb1) of output tile t, piece `idx` of
+// the `count` pieces that together cover the tile's K range.
+struct Work {
+  long long t;
+  int kb0, kb1;
+  int idx, count;
+};
+
+// The sequence of work units one block processes, in the same order for the
+// producer, the MMA issuer and the epilogue.
+struct WorkIter {
+  long long cursor, end, step;
+  __device__ __forceinline__ WorkIter(const KParams& p, long long num_tiles) {
+    if (p.work_mode == 2) {
+      const long long total = num_tiles * p.num_kb;
+      cursor = static_cast<long long>(blockIdx.x) * p.sk_width;
+      end = min(total, cursor + p.sk_width);
+      step = 0;
+    } else {
+      const long long units = p.work_mode == 1 ? num_tiles * p.splits : num_tiles;
+      cursor = blockIdx.x;
+      end = units;
+      step = gridDim.x;
+    }
+  }
+  __device__ __forceinline__ bool next(const KParams& p, Work& w) {
+    if (cursor >= end) return false;
+    if (p.work_mode == 2) {
+      const long long nkb = p.num_kb;
+      w.t = cursor / nkb;
+      w.kb0 = static_cast<int>(cursor - w.t * nkb);
+      w.kb1 = static_cast<int>(min(nkb, static_cast<long long>(w.kb0) + (end - cursor)));
+      const long long first = (w.t * nkb) / p.sk_width;
+      const long long last = ((w.t + 1) * nkb - 1) / p.sk_width;
+      w.idx = static_cast<int>(blockIdx.x - first);
+      w.count = static_cast<int>(last - first + 1);
+      cursor += w.kb1 - w.kb0;
+    } else if (p.work_mode == 1) {
+      w.t = cursor / p.splits;
+      w.idx = static_cast<int>(cursor - w.t * p.splits);
+      w.count = p.splits;
+      w.kb0 = w.idx * p.kb_per_split;
+      w.kb1 = min(w.kb0 + p.kb_per_split, p.num_kb);
+      cursor += step;
+    } else {
+      w.t = cursor;
+      w.idx = 0;
+      w.count = 1;
+      w.kb0 = 0;
+      w.kb1 = p.num_kb;
+      cursor += step;
+    }
+    return true;
+  }
+};
 
 struct SharedCtl {
   int abort;
@@ -143,10 +219,11 @@ __device__ __forceinline__ float from_f32<float>(float v) { return v; }
 
 // Where a tile lives.
 struct TileCoord {
-  int p0;        // first P row (dense: global; grouped: global row of A)
-  int q0;        // first Q row
-  int group;     // grouped: group index (0 otherwise)
-  int row_end;   // grouped: one past the group's last global row
+  int p0;        // first P row (dense: within the batch; grouped: global row of A)
+  int q0;        // first Q block (caller scales by BN)
+  int group;     // grouped: group index; dense: batch index
+  int zp, zq;    // third TMA coordinate of the P and Q copies
+  int row_end;   // one past the last output row this tile may store
   bool valid;
 };
 
@@ -163,10 +240,14 @@ __device__ __forceinline__ TileCoord tile_coord(long long t, const KParams& p, i
   c.group = 0;
   c.valid = true;
   if constexpr (!GROUPED) {
+    const long long b = t / p.tiles_per_batch;
     int pb, qb;
-    raster_tile(t, p.num_p, p.num_q, p.group_m, pb, qb);
+    raster_tile(t - b * p.tiles_per_batch, p.num_p, p.num_q, p.group_m, pb, qb);
     c.p0 = pb * kBM;
     c.q0 = qb;  // caller scales by BN
+    c.group = static_cast<int>(b);
+    c.zp = static_cast<int>(b) * p.z_p;
+    c.zq = static_cast<int>(b) * p.z_q;
     c.row_end = p.M;
   } else {
     // tiles are visited in increasing order by each role, so walk forward
@@ -182,6 +263,8 @@ __device__ __forceinline__ TileCoord tile_coord(long long t, const KParams& p, i
     int mb, nb;
     raster_tile(local, mblocks, num_q_blocks, p.group_m, mb, nb);
     c.group = g;
+    c.zp = 0;
+    c.zq = g;
     c.p0 = gt->row_start[g] + mb * kBM;
     c.q0 = nb;
     c.row_end = min(gt->row_start[g + 1], p.M);
@@ -189,98 +272,71 @@ __device__ __forceinline__ TileCoord tile_coord(long long t, const KParams& p, i
   return c;
 }
 
-// Epilogue for one accumulator row held by this thread: TMEM columns
-// [0, BN) of lane `prow - p0` become output row `prow`, columns q0 .. q0+BN:
-// fp32 -> (+ bias[col]) -> (ReLU) -> round to OutT -> store.  Called by all
-// 32 lanes of an epilogue warp (the TMEM loads are warp-collective); rows at
-// or past row_end and columns at or past N are not stored.
-template <int BN, typename InT, typename OutT>
-__device__ __forceinline__ void store_acc_rows(uint32_t taddr, int prow, int row_end, int q0,
-                                               const KParams& p, const InT* bias_g, bool relu,
-                                               OutT* C) {
-  const bool row_ok = prow < row_end;
-  OutT* crow = C + static_cast<long long>(prow) * p.ldc;
-#pragma unroll 1
-  for (int cc = 0; cc < BN; cc += 32) {
-    const int col0 = q0 + cc;
-    if (col0 >= p.N) break;  // warp-uniform
-    uint32_t v[32];
-    tmem_ld_32x32b_x32(taddr + cc, v);
-    tmem_ld_wait();
-    float f[32];
+
+// Partial tiles are laid out [BN/4][128 rows][4 floats] so that the 32
+// lanes of a warp, which hold 32 consecutive rows, touch 512 contiguous
+// bytes per float4 access.
+
+// Write 16 raw fp32 accumulator values (columns cc .. cc+15 of this thread's
+// row) into a partial tile.
+__device__ __forceinline__ void put_partial16(float* tile, int row, int cc, const uint32_t (&v)[16]) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      float x = __uint_as_float(v[j]);
-      if (bias_g != nullptr && col0 + j < p.N) x += to_f32<InT>(bias_g[col0 + j]);
-      if (relu) x = fmaxf(x, 0.0f);
-      f[j] = x;
-    }
-    if (row_ok) {
-      if (col0 + 32 <= p.N) {
-        if constexpr (sizeof(OutT) == 2) {
-          uint4* dst = reinterpret_cast<uint4*>(crow + col0);
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-            dst[j] = make_uint4(pack2<OutT>(f[8 * j + 0], f[8 * j + 1]),
-                                pack2<OutT>(f[8 * j + 2], f[8 * j + 3]),
-                                pack2<OutT>(f[8 * j + 4], f[8 * j + 5]),
-                                pack2<OutT>(f[8 * j + 6], f[8 * j + 7]));
-        } else {
-          float4* dst = reinterpret_cast<float4*>(crow + col0);
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            dst[j] = make_float4(f[4 * j], f[4 * j + 1], f[4 * j + 2], f[4 * j + 3]);
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          if (col0 + j < p.N) crow[col0 + j] = from_f32<OutT>(f[j]);
-      }
-    }
-  }
+  for (int j = 0; j < 4; ++j)
+    __stcg(reinterpret_cast<float4*>(tile) + (static_cast<long long>(cc / 4 + j) * kBM + row),
+           make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                       __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
 }
 
-// Sum of 16 consecutive fp32 values over `splits` partial tiles `stride`
-// floats apart, in split order (so the result does not depend on which
-// block finished last).
-__device__ __forceinline__ void sum_partials16(const float* src, int splits, long long stride,
-                                               float (&f)[16]) {
+// Columns cc .. cc+15 of this thread's row summed over `count` partial tiles
+// `stride` floats apart, in piece order (so the result does not depend on
+// which block finished last); returned as raw fp32 bits.
+__device__ __forceinline__ void sum_partials16(const float* tile0, long long stride, int count,
+                                               int row, int cc, uint32_t (&out)[16]) {
+  float f[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) f[j] = 0.0f;
-  for (int s = 0; s < splits; ++s) {
-    const float4* q = reinterpret_cast<const float4*>(src + s * stride);
+  for (int s = 0; s < count; ++s) {
+    const float4* q = reinterpret_cast<const float4*>(tile0 + s * stride);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float4 v = __ldcg(q + j);
+      const float4 v = __ldcg(q + (static_cast<long long>(cc / 4 + j) * kBM + row));
       f[4 * j] += v.x;
       f[4 * j + 1] += v.y;
       f[4 * j + 2] += v.z;
       f[4 * j + 3] += v.w;
     }
   }
+#pragma unroll
+  for (int j = 0; j < 16; ++j) out[j] = __float_as_uint(f[j]);
 }
 
-// Split-K finish for one output row: sum the partial rows (row-major
-// [split][128][BN] fp32 starting at `base` for this row), then bias, ReLU,
-// cast and store exactly like store_acc_rows.
-template <int BN, typename InT, typename OutT>
-__device__ __forceinline__ void store_partial_sums(const float* base, int splits, int prow,
-                                                   int row_end, int q0, const KParams& p,
-                                                   const InT* bias_g, bool relu, OutT* C) {
+// Epilogue for one accumulator row held by this thread, from any source of
+// raw fp32 values: src.get<16>(cc, v) fills v[0..15] with columns cc .. cc+15
+// of the row (a warp-collective TMEM load, or a partial-tile sum).  Output row
+// `prow`, columns q0 .. q0+TILE_N: + bias[col] -> ReLU -> round to OutT ->
+// store from registers.  Rows at or past row_end and columns at or past N are
+// not stored.  Called by all 32 lanes of an epilogue warp.
+template <int TILE_N, typename InT, typename OutT, typename Src>
+__device__ __forceinline__ void store_rows_from(Src&& src, int prow, int row_end, int q0,
+                                                const KParams& p, const InT* bias_g, bool relu,
+                                                OutT* C) {
   const bool row_ok = prow < row_end;
   OutT* crow = C + static_cast<long long>(prow) * p.ldc;
-  const long long stride = static_cast<long long>(kBM) * BN;
 #pragma unroll 1
-  for (int cc = 0; cc < BN; cc += 16) {
+  for (int cc = 0; cc < TILE_N; cc += 16) {
     const int col0 = q0 + cc;
-    if (col0 >= p.N || !row_ok) break;
+    if (col0 >= p.N) break;  // warp-uniform
+    uint32_t v[16];
+    src.template get<16>(cc, v);
     float f[16];
-    sum_partials16(base + cc, splits, stride, f);
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      if (bias_g != nullptr && col0 + j < p.N) f[j] += to_f32<InT>(bias_g[col0 + j]);
-      if (relu) f[j] = fmaxf(f[j], 0.0f);
+      float x = __uint_as_float(v[j]);
+      if (bias_g != nullptr && col0 + j < p.N) x += to_f32<InT>(bias_g[col0 + j]);
+      if (relu) x = fmaxf(x, 0.0f);
+      f[j] = x;
     }
+    if (!row_ok) continue;
     if (col0 + 16 <= p.N) {
       if constexpr (sizeof(OutT) == 2) {
         uint4* dst = reinterpret_cast<uint4*>(crow + col0);
@@ -303,5 +359,142 @@ __device__ __forceinline__ void store_partial_sums(const float* base, int splits
     }
   }
 }
+
+// Bytes of the epilogue staging area: 4 epilogue warps x 2 buffers x one
+// 32-row box of 128-byte rows (4 KB).
+constexpr uint32_t kEpiStageBytes = 4 * 2 * 4096;
+
+// Epilogue through shared memory and TMA stores, for one warp's 32
+// accumulator rows (TMEM lanes of this warp's quadrant, output rows
+// row0 .. row0+31) and output columns q0 .. q0+TILE_N.  Each pass takes 128
+// bytes of every row (64 16-bit or 32 fp32 outputs): TMEM -> registers ->
+// bias, ReLU, round -> a 128B-swizzled 32 x 128 B staging buffer (16-byte
+// chunk c of row r at chunk c ^ (r % 8), so the eight rows of a store phase hit
+// eight different bank groups) -> one lane issues a TMA store of the box (at
+// batch z of the 3-D output map), which clips rows >= M and columns >= N.  Two buffers per warp alternate;
+// `count` carries the warp's store count across tiles.  Called by all 32
+// lanes of the warp.
+template <int TILE_N, typename InT, typename OutT, typename Src>
+__device__ __forceinline__ void store_tma_from(Src&& src, int row0, int q0, int z,
+                                               const KParams& p, const InT* bias, bool relu,
+                                               uint32_t stage, uint32_t& count,
+                                               const CUtensorMap* tmC) {
+  constexpr int CH = 128 / static_cast<int>(sizeof(OutT));  // outputs per 128-byte row chunk
+  const int lane = threadIdx.x & 31;
+  // a box must start inside the tensor: a slab wholly below the last row
+  // stores nothing (warp-uniform)
+  if (row0 >= p.M) return;
+#pragma unroll 1
+  for (int c0 = 0; c0 < TILE_N; c0 += CH) {
+    const int col0 = q0 + c0;
+    if (col0 >= p.N) break;  // warp-uniform
+    uint32_t v[CH];
+    src.template get<CH>(c0, v);
+    uint32_t packed[32];
+    if constexpr (sizeof(OutT) == 2) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float x0 = __uint_as_float(v[2 * j]), x1 = __uint_as_float(v[2 * j + 1]);
+        if (bias != nullptr) {
+          if (col0 + 2 * j < p.N) x0 += to_f32<InT>(bias[col0 + 2 * j]);
+          if (col0 + 2 * j + 1 < p.N) x1 += to_f32<InT>(bias[col0 + 2 * j + 1]);
+        }
+        if (relu) {
+          x0 = fmaxf(x0, 0.0f);
+          x1 = fmaxf(x1, 0.0f);
+        }
+        packed[j] = pack2<OutT>(x0, x1);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float x = __uint_as_float(v[j]);
+        if (bias != nullptr && col0 + j < p.N) x += to_f32<InT>(bias[col0 + j]);
+        if (relu) x = fmaxf(x, 0.0f);
+        packed[j] = __float_as_uint(x);
+      }
+    }
+    // the buffer written two stores ago must have been read by its TMA store
+    if (count >= 2) {
+      if (lane == 0) tma_store_wait_read<1>();
+      __syncwarp();
+    }
+    const uint32_t buf = stage + (count & 1u) * 4096u;
+    const uint32_t row_addr = buf + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t dst = row_addr + ((static_cast<uint32_t>(c) ^ (lane & 7u)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[4 * c]),
+                   "r"(packed[4 * c + 1]), "r"(packed[4 * c + 2]), "r"(packed[4 * c + 3])
+                   : "memory");
+    }
+    fence_proxy_async_shared();  // these generic writes -> the TMA (async proxy) read
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(tmC, buf, col0, row0, z);
+      tma_store_commit();
+    }
+    ++count;
+  }
+}
+
+// TMEM as a source of raw accumulator values for the epilogues above: the
+// warp's 32 lanes x 16 consecutive columns starting at `taddr + cc`.
+// get<W>(cc, v) fills v with W consecutive columns starting at cc; all
+// loads of one call are in flight together and waited for once.
+// With nacc > 1 the values are the in-order sum of nacc accumulators that
+// sit acc_stride columns apart.
+struct TmemSrc {
+  uint32_t taddr;
+  int nacc = 1;
+  int acc_stride = 0;
+  template <int W>
+  __device__ __forceinline__ void get(int cc, uint32_t (&v)[W]) const {
+    static_assert(W % 16 == 0, "whole 16-column groups");
+    if (nacc > 1) {  // warp-uniform
+#pragma unroll
+      for (int h = 0; h < W; h += 16) {
+        float f[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) f[j] = 0.0f;
+        for (int r = 0; r < nacc; ++r) {
+          uint32_t u[16];
+          tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(cc + h + r * acc_stride), u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) f[j] += __uint_as_float(u[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[h + j] = __float_as_uint(f[j]);
+      }
+      return;
+    }
+    if constexpr (W % 32 == 0) {
+#pragma unroll
+      for (int h = 0; h < W; h += 32)
+        tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(cc + h),
+                           *reinterpret_cast<uint32_t(*)[32]>(&v[h]));
+    } else {
+#pragma unroll
+      for (int h = 0; h < W; h += 16)
+        tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(cc + h),
+                           *reinterpret_cast<uint32_t(*)[16]>(&v[h]));
+    }
+    tmem_ld_wait();
+  }
+};
+
+// A partial-tile sum as a source (the last piece of a split tile).
+struct PartialSrc {
+  const float* tile0;
+  long long stride;
+  int count, row;
+  template <int W>
+  __device__ __forceinline__ void get(int cc, uint32_t (&v)[W]) const {
+#pragma unroll
+    for (int h = 0; h < W; h += 16)
+      sum_partials16(tile0, stride, count, row, cc + h, *reinterpret_cast<uint32_t(*)[16]>(&v[h]));
+  }
+};
 
 }  // namespace dg16

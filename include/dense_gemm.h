@@ -104,6 +104,30 @@ GEMM_API int gemm(int M, int N, int K, const void* A, int64_t lda, const void* B
          int64_t ldc, const void* bias, unsigned epilogue, int dtype, void* stream);
 
 /*
+ * gemm_strided_batched -- `batch` independent GEMMs in one launch
+ * ("用Triton跨芯片优化GEMM" section 4.3 benchmarks single and multi-batch
+ * GEMMs).  For b in [0, batch):
+ *     C_b = act(A_b . B_b + bias_b),  X_b = X + b*stride_x  (elements)
+ * with every other argument as in gemm() (one lda/ldb/ldc, one layout flag,
+ * one dtype for all batches).  gemm() is this call with batch = 1.
+ *
+ *   batch      >= 0; 0 is a no-op
+ *   stride_a   0 (every batch reads the same A) or >= lda*M
+ *   stride_b   0 (shared B) or >= ldb*K (row-major) / ldb*N (column-major)
+ *   stride_c   >= ldc*M: outputs never overlap
+ *   stride_bias 0 (one bias vector for all batches) or the distance between
+ *              the batches' length-N bias vectors
+ * stride_a*2, stride_b*2 and stride_c*sizeof(output) must be multiples of 16
+ * bytes when batch > 1 (else GEMM_ERR_MISALIGNED); a stride that breaks the
+ * rules above returns GEMM_ERR_INVALID_ARG.  With batch == 1 the strides are
+ * ignored.
+ */
+GEMM_API int gemm_strided_batched(int batch, int M, int N, int K, const void* A, int64_t lda,
+                                  int64_t stride_a, const void* B, int64_t ldb, int64_t stride_b,
+                                  void* C, int64_t ldc, int64_t stride_c, const void* bias,
+                                  int64_t stride_bias, unsigned epilogue, int dtype, void* stream);
+
+/*
  * grouped_gemm -- the per-expert GEMMs of an MoE layer in one launch
  * ("用Triton跨芯片优化GEMM" section 2.3: a MoE layer runs dozens of GEMMs).
  *

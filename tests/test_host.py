@@ -166,3 +166,22 @@ def test_valid_call_without_a_device_reports_cuda_error():
     L = dg.lib()
     assert L.gemm(4, 4, 4, P, 8, P, 8, P, 8, None, 0, 0, None) == dg.GEMM_ERR_CUDA
     assert L.gemm_device_status(None, 0) == dg.GEMM_ERR_CUDA
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (batch, M, N, K, A, lda, sA, B, ldb, sB, C, ldc, sC, bias, sbias, epi, dtype)
+    ((-1, 4, 8, 8, P, 8, 64, P, 8, 64, P, 8, 32, None, 0, 0, 0), dg.GEMM_ERR_INVALID_ARG),
+    ((2, 4, 8, 8, P, 8, 16, P, 8, 64, P, 8, 32, None, 0, 0, 0), dg.GEMM_ERR_INVALID_ARG),   # A overlaps
+    ((2, 4, 8, 8, P, 8, 32, P, 8, 40, P, 8, 32, None, 0, 0, 0), dg.GEMM_ERR_INVALID_ARG),   # B overlaps
+    ((2, 4, 8, 8, P, 8, 32, P, 8, 64, P, 8, 24, None, 0, 0, 0), dg.GEMM_ERR_INVALID_ARG),   # C overlaps
+    ((2, 4, 8, 8, P, 8, 36, P, 8, 64, P, 8, 32, None, 0, 0, 0), dg.GEMM_ERR_MISALIGNED),    # sA*2 % 16
+    ((2, 4, 8, 8, P, 8, 32, P, 8, 64, P, 8, 36, None, 0, 0, 0), dg.GEMM_ERR_MISALIGNED),    # sC*2 % 16
+    ((2, 4, 8, 8, P, 8, 32, P, 8, 64, P, 8, 32, None, -8, 0, 0), dg.GEMM_ERR_INVALID_ARG),  # sbias < 0
+])
+def test_batched_argument_errors(args, expect):
+    assert dg.lib().gemm_strided_batched(*args, None) == expect
+
+
+def test_batched_empty_is_a_noop():
+    assert dg.lib().gemm_strided_batched(0, 4, 4, 4, P, 8, 32, P, 8, 32, P, 8, 32, None, 0, 0, 0,
+                                         None) == 0

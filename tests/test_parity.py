@@ -73,7 +73,7 @@ def test_moe_grouped_sampled():
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("b_col", [False, True])
-@pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 18])
+@pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 12, 13, 23, 24])
 def test_exact_integers(dtype, b_col, config):
     """Integer inputs in [-2, 2] with K <= 4096: every partial sum is an
     exact integer below 2^24, so the fp32 accumulator is exact in any order
@@ -144,7 +144,7 @@ def test_empty_m_or_n_is_a_noop():
     assert bool((g.ibuf.cpu() == g.sent).all())
 
 
-@pytest.mark.parametrize("config", range(21))
+@pytest.mark.parametrize("config", range(25))
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("out_f32", [False, True])
 def test_every_config_on_ragged_problem(config, dtype, out_f32):
@@ -263,7 +263,8 @@ def test_watchdog_times_out_cleanly_and_context_survives():
 # --------------------------------------------------------------- split-K
 
 def _split_configs():
-    return [i for i in range(dg.gemm_num_configs()) if "_k" in dg.gemm_config_name(i)]
+    return [i for i in range(dg.gemm_num_configs())
+            if "_k" in dg.gemm_config_name(i) or dg.gemm_config_name(i).endswith("_sk")]
 
 
 @pytest.mark.parametrize("swap", [False, True])
@@ -312,3 +313,110 @@ def test_split_k_on_concurrent_streams():
     for A, o in zip(As, outs):
         ref = oracle.gemm(M, N, K, A, K, B, N, threads=THREADS)
         compare(o.double().cpu().numpy(), ref, 2, "split-K on a side stream")
+
+
+# ------------------------------------------------------- strided batches
+
+class BatchGuard:
+    """`batch` outputs M x N (leading dimension ldc) stride_c elements apart
+    in one sentinel-filled buffer: the gaps between batches and the ldc
+    padding must stay untouched."""
+
+    def __init__(self, batch, M, N, ldc, stride_c, dtype, pad=128):
+        self.b, self.M, self.N, self.ldc, self.sc, self.pad = batch, M, N, ldc, stride_c, pad
+        self.buf = torch.empty(pad + batch * stride_c + pad, dtype=dtype, device="cuda")
+        self.ibuf = self.buf.view(torch.int32 if dtype == torch.float32 else torch.int16)
+        from gpu_helpers import _SENT16, _SENT32
+        self.sent = _SENT32 if dtype == torch.float32 else _SENT16
+        self.ibuf.fill_(self.sent)
+        self.ptr = self.buf.data_ptr() + pad * self.buf.element_size()
+
+    def matrix(self, b):
+        o = self.pad + b * self.sc
+        return self.buf[o:o + self.M * self.ldc].view(self.M, self.ldc)[:, :self.N]
+
+    def check_canaries(self):
+        raw = self.ibuf.cpu()
+        mask = torch.ones_like(raw, dtype=torch.bool)
+        for b in range(self.b):
+            o = self.pad + b * self.sc
+            body = mask[o:o + self.M * self.ldc].view(self.M, self.ldc)
+            body[:, :self.N] = False
+        assert bool((raw[mask] == self.sent).all()), "write outside the batch outputs"
+
+
+@pytest.mark.parametrize("config", [None, 0, 1, 4, 13, 8, 23, 2])
+@pytest.mark.parametrize("b_col", [False, True])
+@pytest.mark.parametrize("share", ["none", "a", "b"])
+def test_strided_batched(config, b_col, share):
+    name = dg.gemm_config_name(config) if config is not None else "table"
+    if name.startswith("swap") and not b_col:
+        pytest.skip("swapped tiles need column-major B")
+    batch = 3
+    M, N, K = (20 if name.startswith("swap") else 300), 264, 200
+    gen = torch.Generator().manual_seed(4000 + (config or 0) + 7 * b_col)
+    lda, ldb, ldc = K + 8, (K + 16 if b_col else N + 8), N + 8
+    sa = 0 if share == "a" else M * lda + 64
+    sb = 0 if share == "b" else (N if b_col else K) * ldb + 32
+    sc, sbias = M * ldc + 96, N + 8
+    A = torch.randn(max(1, batch if sa else 1), M, K, generator=gen).half()
+    B = torch.randn(max(1, batch if sb else 1), *((N, K) if b_col else (K, N)), generator=gen).half()
+    bias = torch.randn(batch, N, generator=gen).half()
+    # device buffers with the requested strides (padding NaN-filled)
+    dA = torch.full((max(1, batch if sa else 1) * max(sa, M * lda) + 64,), float("nan"),
+                    dtype=torch.half, device="cuda")
+    dB = torch.full((max(1, batch if sb else 1) * max(sb, B.shape[1] * ldb) + 64,), float("nan"),
+                    dtype=torch.half, device="cuda")
+    for i in range(A.shape[0]):
+        dA[i * sa:i * sa + M * lda].view(M, lda)[:, :K] = A[i].cuda()
+    for i in range(B.shape[0]):
+        r, c = B.shape[1], B.shape[2]
+        dB[i * sb:i * sb + r * ldb].view(r, ldb)[:, :c] = B[i].cuda()
+    dbias = torch.zeros(batch * sbias, dtype=torch.half, device="cuda")
+    for i in range(batch):
+        dbias[i * sbias:i * sbias + N] = bias[i].cuda()
+    g = BatchGuard(batch, M, N, ldc, sc, torch.float16)
+    epi = dg.GEMM_EPI_BIAS | dg.GEMM_EPI_RELU | (dg.GEMM_B_COL_MAJOR if b_col else 0)
+    if config is not None:
+        assert dg.gemm_force_config(config) == 0
+    try:
+        rc = dg.gemm_strided_batched(batch, M, N, K, dA, lda, sa, dB, ldb, sb, g.ptr, ldc, sc,
+                                     dbias, sbias, epi, dg.GEMM_F16)
+    finally:
+        dg.gemm_force_config(-1)
+    assert rc == 0, dg.gemm_status_string(rc)
+    torch.cuda.synchronize()
+    assert dg.gemm_device_status() == 0
+    for i in range(batch):
+        Ai = A[i if sa else 0]
+        Bi = B[i if sb else 0]
+        ref = oracle.gemm(M, N, K, Ai, K, Bi, K if b_col else N, b_colmajor=b_col, bias=bias[i],
+                          relu=True, threads=THREADS)
+        compare(g.matrix(i).double().cpu().numpy(), ref, 2, f"{name} batch {i}")
+    g.check_canaries()
+
+
+def test_batched_k_zero_and_shared_bias():
+    batch, M, N = 2, 5, 24
+    bias = torch.linspace(-2, 2, N).half()
+    g = BatchGuard(batch, M, N, N, M * N + 40, torch.float16)
+    rc = dg.gemm_strided_batched(batch, M, N, 0, None, 0, 0, None, 0, 0, g.ptr, N, M * N + 40,
+                                 bias.cuda(), 0, dg.GEMM_EPI_BIAS | dg.GEMM_EPI_RELU, dg.GEMM_F16)
+    assert rc == 0
+    torch.cuda.synchronize()
+    ref = oracle.gemm(M, N, 0, None, 0, None, 0, bias=bias, relu=True)
+    for i in range(batch):
+        compare(g.matrix(i).double().cpu().numpy(), ref, 2, "K=0 batch")
+    g.check_canaries()
+
+
+def test_bmm_helper_matches_torch_layouts():
+    gen = torch.Generator().manual_seed(9)
+    a = torch.randn(4, 130, 96, generator=gen).bfloat16().cuda()
+    b = torch.randn(4, 96, 72, generator=gen).bfloat16().cuda()
+    out = dg.bmm(a, b)
+    torch.cuda.synchronize()
+    for i in range(4):
+        ref = oracle.gemm(130, 72, 96, a[i].cpu(), 96, b[i].cpu(), 72, dtype="bf16",
+                          threads=THREADS)
+        compare(out[i].double().cpu().numpy(), ref, 2, "bmm")
