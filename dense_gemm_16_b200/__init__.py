@@ -29,7 +29,7 @@ GEMM_ERR_MISALIGNED = -3
 GEMM_ERR_CUDA = -4
 GEMM_ERR_DEVICE_TIMEOUT = -5
 
-GEMM_F16, GEMM_BF16, GEMM_F16_OUT_F32, GEMM_BF16_OUT_F32 = 0, 1, 2, 3
+GEMM_F16, GEMM_BF16, GEMM_F16_OUT_F32, GEMM_BF16_OUT_F32, GEMM_F32_TF32 = 0, 1, 2, 3, 4
 GEMM_EPI_BIAS = 0x1
 GEMM_EPI_RELU = 0x2
 GEMM_B_COL_MAJOR = 0x100
@@ -198,6 +198,8 @@ def dtype_code(in_dtype, out_f32: bool = False) -> int:
         return GEMM_F16_OUT_F32 if out_f32 else GEMM_F16
     if in_dtype == torch.bfloat16:
         return GEMM_BF16_OUT_F32 if out_f32 else GEMM_BF16
+    if in_dtype == torch.float32:  # multiplied as tf32, fp32 out
+        return GEMM_F32_TF32
     raise TypeError(f"unsupported input dtype {in_dtype}")
 
 
@@ -213,7 +215,8 @@ def matmul(a, b, bias=None, relu: bool = False, b_col_major: bool = False, out=N
     N = b.shape[0] if b_col_major else b.shape[1]
     code = dtype_code(a.dtype, out_f32)
     if out is None:
-        out = torch.empty(M, N, device=a.device, dtype=torch.float32 if out_f32 else a.dtype)
+        out = torch.empty(M, N, device=a.device,
+                          dtype=torch.float32 if (out_f32 or code == GEMM_F32_TF32) else a.dtype)
     epi = (GEMM_EPI_BIAS if bias is not None else 0) | (GEMM_EPI_RELU if relu else 0) | \
         (GEMM_B_COL_MAJOR if b_col_major else 0)
     rc = gemm(M, N, K, a, a.stride(0), b, b.stride(0), out, out.stride(0), bias, epi, code,

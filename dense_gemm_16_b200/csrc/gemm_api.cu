@@ -180,7 +180,8 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 // A 2- or 3-D tensor map with 128-byte swizzle and zero fill outside the
 // tensor.  dims[0] is the contiguous dimension; strides in bytes.
 int make_map_t(CUtensorMap* m, const void* base, CUtensorMapDataType type, int rank,
-               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto enc = encoder();
   if (!enc) return GEMM_ERR_CUDA;
   cuuint64_t gd[3], gs[2];
@@ -191,7 +192,7 @@ int make_map_t(CUtensorMap* m, const void* base, CUtensorMapDataType type, int r
   }
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
   CUresult r = enc(m, type, rank, const_cast<void*>(base), gd, gs, bx, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? GEMM_OK : GEMM_ERR_CUDA;
 }
@@ -219,8 +220,20 @@ int make_c_map(CUtensorMap* m, void* C, int M, int N, int64_t ldc, int dtype) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int out_bytes(int dtype) { return (dtype == GEMM_F16_OUT_F32 || dtype == GEMM_BF16_OUT_F32) ? 4 : 2; }
+int out_bytes(int dtype) {
+  return (dtype == GEMM_F16_OUT_F32 || dtype == GEMM_BF16_OUT_F32 || dtype == GEMM_F32_TF32) ? 4
+                                                                                             : 2;
+}
 bool in_bf16(int dtype) { return dtype == GEMM_BF16 || dtype == GEMM_BF16_OUT_F32; }
+bool in_tf32(int dtype) { return dtype == GEMM_F32_TF32; }
+int in_bytes(int dtype) { return in_tf32(dtype) ? 4 : 2; }
+// K elements per ring stage: one 128-byte swizzle row
+int kb_elems(int dtype) { return 128 / in_bytes(dtype); }
+CUtensorMapDataType in_map_type(int dtype) {
+  return in_tf32(dtype) ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                        : (in_bf16(dtype) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                          : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+}
 
 // Checks shared by gemm() and grouped_gemm() once sizes are known.
 int check_common(int N, int K, const void* A, int64_t lda, const void* B, int64_t ldb, void* C,
@@ -229,24 +242,33 @@ int check_common(int N, int K, const void* A, int64_t lda, const void* B, int64_
   if ((epi & GEMM_EPI_BIAS) && !bias) return GEMM_ERR_INVALID_ARG;
   if (ldc < N) return GEMM_ERR_INVALID_ARG;
   if (!aligned16(C) || (ldc * out_bytes(dtype)) % 16 != 0) return GEMM_ERR_MISALIGNED;
-  if ((epi & GEMM_EPI_BIAS) && (reinterpret_cast<uintptr_t>(bias) & 1u)) return GEMM_ERR_MISALIGNED;
+  if ((epi & GEMM_EPI_BIAS) &&
+      (reinterpret_cast<uintptr_t>(bias) & static_cast<uintptr_t>(in_bytes(dtype) - 1)))
+    return GEMM_ERR_MISALIGNED;
   if (K > 0) {
     if (!A || !B) return GEMM_ERR_INVALID_ARG;
     const bool bcol = (epi & GEMM_B_COL_MAJOR) != 0;
     if (lda < K || ldb < (bcol ? K : N)) return GEMM_ERR_INVALID_ARG;
-    if (!aligned16(A) || !aligned16(B) || lda % 8 != 0 || ldb % 8 != 0) return GEMM_ERR_MISALIGNED;
+    const int per16 = 16 / in_bytes(dtype);  // elements per 16 bytes
+    if (!aligned16(A) || !aligned16(B) || lda % per16 != 0 || ldb % per16 != 0)
+      return GEMM_ERR_MISALIGNED;
   }
   return GEMM_OK;
 }
 
 int check_dtype_epi(unsigned epi, int dtype) {
-  if (dtype < GEMM_F16 || dtype > GEMM_BF16_OUT_F32) return GEMM_ERR_UNSUPPORTED;
+  if (dtype < GEMM_F16 || dtype > GEMM_F32_TF32) return GEMM_ERR_UNSUPPORTED;
   if (epi & ~kEpiMask) return GEMM_ERR_UNSUPPORTED;
   return GEMM_OK;
 }
 
 // The kernel instance for a config and problem variant.
-KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool grouped) {
+KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool grouped,
+                       bool tf32 = false) {
+  if (tf32) {  // fp32 inputs: single-CTA dense tiles only
+    if (c.kind != kKindSingle || grouped) return {nullptr, 0};
+    return kernels_tf32(c.bn, q_mn);
+  }
   if (c.kind == kKindSwap) {
     if (q_mn || grouped) return {nullptr, 0};  // needs column-major B
     return kernels_swap(c.bn, bf16, f32);
@@ -318,7 +340,8 @@ int check_batch(const DenseProblem& d) {
   if (d.K > 0) {
     if (d.stride_a != 0 && d.stride_a < ext_a) return GEMM_ERR_INVALID_ARG;
     if (d.stride_b != 0 && d.stride_b < ext_b) return GEMM_ERR_INVALID_ARG;
-    if ((d.stride_a * 2) % 16 != 0 || (d.stride_b * 2) % 16 != 0) return GEMM_ERR_MISALIGNED;
+    const int ib = in_bytes(d.dtype);
+    if ((d.stride_a * ib) % 16 != 0 || (d.stride_b * ib) % 16 != 0) return GEMM_ERR_MISALIGNED;
   }
   if (d.stride_c < d.ldc * d.M) return GEMM_ERR_INVALID_ARG;
   if ((d.stride_c * out_bytes(d.dtype)) % 16 != 0) return GEMM_ERR_MISALIGNED;
@@ -339,6 +362,7 @@ int launch_fill(const DenseProblem& d, cudaStream_t stream) {
 
 int fill_dispatch(const DenseProblem& d, cudaStream_t stream) {
   switch (d.dtype) {
+    case GEMM_F32_TF32: return launch_fill<float, float>(d, stream);
     case GEMM_F16: return launch_fill<__half, __half>(d, stream);
     case GEMM_BF16: return launch_fill<__nv_bfloat16, __nv_bfloat16>(d, stream);
     case GEMM_F16_OUT_F32: return launch_fill<__half, float>(d, stream);
@@ -362,10 +386,14 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   const int M = d.M, N = d.N, K = d.K;
   const bool bcol = (d.epi & GEMM_B_COL_MAJOR) != 0;
   const bool bf16 = in_bf16(d.dtype);
+  const bool tf32 = in_tf32(d.dtype);
   const bool f32 = out_bytes(d.dtype) == 4;
   const bool swap = cfg.kind == kKindSwap;
   const bool pair = cfg.kind == kKindPair;
-  const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false);
+  const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false, tf32);
+  const int ib = in_bytes(d.dtype);
+  const uint32_t kbe = static_cast<uint32_t>(kb_elems(d.dtype));  // K per stage
+  const CUtensorMapDataType it = in_map_type(d.dtype);
   if (!k.fn || (swap && !bcol)) return GEMM_ERR_UNSUPPORTED;
 
   // batch extents of the 3-D maps: a shared operand has one batch
@@ -373,8 +401,8 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   const uint64_t nb_a = (bat && d.stride_a) ? d.batch : 1, nb_b = (bat && d.stride_b) ? d.batch : 1;
   const uint64_t sa = (bat && d.stride_a) ? d.stride_a : d.lda * M;
   const uint64_t sb = (bat && d.stride_b) ? d.stride_b : (bcol ? d.ldb * N : d.ldb * K);
-  const uint64_t str_a[2] = {static_cast<uint64_t>(d.lda) * 2, sa * 2};
-  const uint64_t str_b[2] = {static_cast<uint64_t>(d.ldb) * 2, sb * 2};
+  const uint64_t str_a[2] = {static_cast<uint64_t>(d.lda) * ib, sa * ib};
+  const uint64_t str_b[2] = {static_cast<uint64_t>(d.ldb) * ib, sb * ib};
 
   CUtensorMap tp, tq, tc;
   std::memset(&tc, 0, sizeof(tc));  // swapped tiles store from registers
@@ -398,7 +426,7 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   kp.M = M;
   kp.N = N;
   kp.K = K;
-  kp.num_kb = (K + kBK - 1) / kBK;
+  kp.num_kb = static_cast<int>((K + kbe - 1) / kbe);
   kp.group_m = cfg.group_m;
   kp.C = d.C;
   kp.ldc = d.ldc;
@@ -410,8 +438,8 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   kp.stride_bias = bat ? d.stride_bias : 0;
   if (!swap) {
     const uint64_t dA[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M), nb_a};
-    const uint32_t bA[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM), 1u};
-    rc = make_map(&tp, d.A, bf16, 3, dA, str_a, bA);
+    const uint32_t bA[3] = {kbe, static_cast<uint32_t>(kBM), 1u};
+    rc = make_map_t(&tp, d.A, it, 3, dA, str_a, bA);
     if (rc) return rc;
     if (bcol) {
       // the pair kernel's CTAs each load half of the tile's B columns
@@ -419,12 +447,15 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
       const uint64_t dB[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), nb_b};
       const uint32_t rows_b = pair ? static_cast<uint32_t>(std::min(cfg.bn, 256) / 2)
                                    : static_cast<uint32_t>(cfg.bn);
-      const uint32_t bB[3] = {static_cast<uint32_t>(kBK), rows_b, 1u};
-      rc = make_map(&tq, d.B, bf16, 3, dB, str_b, bB);
+      const uint32_t bB[3] = {kbe, rows_b, 1u};
+      rc = make_map_t(&tq, d.B, it, 3, dB, str_b, bB);
     } else {
+      // MN-major B: boxes one 128-byte row of N wide, one stage of K deep
+      // (MN-major tf32 must use the 128-byte swizzle with 32-byte atoms)
       const uint64_t dB[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K), nb_b};
-      const uint32_t bB[3] = {64u, static_cast<uint32_t>(kBK), 1u};
-      rc = make_map(&tq, d.B, bf16, 3, dB, str_b, bB);
+      const uint32_t bB[3] = {static_cast<uint32_t>(128 / ib), kbe, 1u};
+      rc = make_map_t(&tq, d.B, it, 3, dB, str_b, bB,
+                      tf32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B);
     }
     if (rc) return rc;
     const int rows_per_tile = pair ? 2 * kBM : kBM;
@@ -435,12 +466,12 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   } else {
     // P = B stored N x K, Q = A (M x K); the accumulator is C^T
     const uint64_t dB[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N), nb_b};
-    const uint32_t bB[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM), 1u};
-    rc = make_map(&tp, d.B, bf16, 3, dB, str_b, bB);
+    const uint32_t bB[3] = {kbe, static_cast<uint32_t>(kBM), 1u};
+    rc = make_map_t(&tp, d.B, it, 3, dB, str_b, bB);
     if (rc) return rc;
     const uint64_t dA[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M), nb_a};
-    const uint32_t bA[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn), 1u};
-    rc = make_map(&tq, d.A, bf16, 3, dA, str_a, bA);
+    const uint32_t bA[3] = {kbe, static_cast<uint32_t>(cfg.bn), 1u};
+    rc = make_map_t(&tq, d.A, it, 3, dA, str_a, bA);
     if (rc) return rc;
     kp.num_p = (N + kBM - 1) / kBM;
     kp.num_q = (M + cfg.bn - 1) / cfg.bn;
@@ -566,8 +597,13 @@ int gemm_strided_batched(int batch, int M, int N, int K, const void* A, int64_t 
   rc = device_state(&ds);
   if (rc) return rc;
   if (K == 0) return fill_dispatch(d, stream);
-  const int cid = select_config(M, N, K, epilogue, false);
+  int cid = select_config(M, N, K, epilogue, false);
   if (cid < 0 || cid >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
+  if (in_tf32(dtype) && kConfigs[cid].kind != kKindSingle && g_forced_config.load() < 0) {
+    // fp32 inputs run on the single-CTA tf32 kernels only
+    const long long tiles256 = static_cast<long long>((M + 127) / 128) * ((N + 255) / 256);
+    cid = (N <= 128 || tiles256 < 96) ? 1 : 0;
+  }
   return run_dense(ds, d, kConfigs[cid], kConfigs[cid].splits, nullptr, stream);
 }
 
@@ -594,6 +630,7 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
   DeviceState* ds = nullptr;
   rc = device_state(&ds);
   if (rc) return rc;
+  if (in_tf32(dtype)) return GEMM_ERR_UNSUPPORTED;  // grouped runs 16-bit inputs only
   const bool bf16 = in_bf16(dtype);
   const bool f32 = out_bytes(dtype) == 4;
   if (K == 0) {

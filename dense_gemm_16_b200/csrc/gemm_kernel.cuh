@@ -38,19 +38,28 @@ namespace dg16 {
 //   STAGES  depth of the operand ring
 //   Q_MN    Q operand is MN-major in memory (row-major B)
 //   IN_BF16 inputs are bf16 (else fp16); InT is the matching CUDA type
+//   TF32    inputs are fp32, multiplied as tf32 (tcgen05 kind::tf32); one
+//           128-byte swizzle row then holds 32 elements instead of 64
 //   OutT    output element type (__half, __nv_bfloat16 or float)
 //   SWAP    P = B (N x K), Q = A: the accumulator holds C^T
 //   GROUPED grouped GEMM (Q tensor map is 3-D: [group][rows][K or N])
-template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT, bool SWAP, bool GROUPED>
+template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT, bool SWAP, bool GROUPED,
+          bool TF32 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmC, const KParams p) {
-  using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
+  using InT = typename std::conditional<
+      TF32, float, typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type>::type;
+  constexpr int ELEM = TF32 ? 4 : 2;           // input bytes
+  constexpr int KB_EL = 128 / ELEM;            // K elements per stage (one swizzle row)
+  constexpr int MN_CHUNK = 128 / ELEM;         // MN elements per MN-major box row
+  constexpr int MMA_K = 32 / ELEM;             // K per MMA instruction (32 bytes)
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N must be 16..256, step 16");
-  static_assert(!Q_MN || BN % 64 == 0, "MN-major Q tiles are whole 64-element swizzle rows");
+  static_assert(!Q_MN || BN % (128 / (TF32 ? 4 : 2)) == 0,
+                "MN-major Q tiles are whole 128-byte swizzle rows");
   static_assert(!(SWAP && GROUPED), "grouped GEMM uses the plain operand order");
-  constexpr uint32_t P_BYTES = kBM * kBK * 2;
-  constexpr uint32_t Q_BYTES = BN * kBK * 2;
+  constexpr uint32_t P_BYTES = kBM * 128;     // 128 rows x one 128-byte K row
+  constexpr uint32_t Q_BYTES = BN * 128;
   constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
   // Swapped (skinny) tiles have a tiny MMA-N, so one accumulator would chain
   // every MMA of a tile through its latency: consecutive K blocks rotate over
@@ -59,7 +68,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int ACC_COLS = NACC * BN;  // TMEM columns per accumulator buffer
   constexpr uint32_t TMEM_COLS = (2 * ACC_COLS <= 32) ? 32 : (2 * ACC_COLS <= 64) ? 64
                                  : (2 * ACC_COLS <= 128) ? 128 : (2 * ACC_COLS <= 256) ? 256 : 512;
-  constexpr uint32_t IDESC = f16_idesc(kBM, BN, IN_BF16 ? 1u : 0u, 0u, Q_MN ? 1u : 0u);
+  constexpr uint32_t IDESC =
+      TF32 ? mma_idesc(kBM, BN, 2u, Q_MN ? 1u : 0u) : f16_idesc(kBM, BN, IN_BF16 ? 1u : 0u, 0u, Q_MN ? 1u : 0u);
   // dense tiles store through shared memory and TMA; grouped tiles must not
   // write past their group's last row and swapped tiles are transposed, so
   // those store from registers
@@ -166,18 +176,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = smem_u32(&full_bar[s]);
           mbar_arrive_expect_tx(fb, STAGE_BYTES);
           if constexpr (GROUPED)
-            tma_load_2d(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, c.p0, fb, pol_p);
+            tma_load_2d(smem_u32(sP + s * P_BYTES), &tmP, kb * KB_EL, c.p0, fb, pol_p);
           else
-            tma_load_3d(smem_u32(sP + s * P_BYTES), &tmP, kb * kBK, c.p0, c.zp, fb, pol_p);
+            tma_load_3d(smem_u32(sP + s * P_BYTES), &tmP, kb * KB_EL, c.p0, c.zp, fb, pol_p);
           const uint32_t qdst = smem_u32(sQ + s * Q_BYTES);
           // Q is 3-D: [group][rows][cols] (grouped) or [batch][rows][cols]
           if constexpr (Q_MN) {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_3d(qdst + j * (64 * kBK * 2), &tmQ, q0 + 64 * j, kb * kBK, c.zq, fb,
-                          pol_q);
+            for (int j = 0; j < BN / MN_CHUNK; ++j)
+              tma_load_3d(qdst + j * (KB_EL * 128), &tmQ, q0 + MN_CHUNK * j, kb * KB_EL, c.zq,
+                          fb, pol_q);
           } else {
-            tma_load_3d(qdst, &tmQ, kb * kBK, q0, c.zq, fb, pol_q);
+            tma_load_3d(qdst, &tmQ, kb * KB_EL, q0, c.zq, fb, pol_q);
           }
         }
       }
@@ -219,15 +229,21 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t pbase = smem_u32(sP + s * P_BYTES);
           const uint32_t qbase = smem_u32(sQ + s * Q_BYTES);
 #pragma unroll
-          for (int k = 0; k < kBK / 16; ++k) {
+          for (int k = 0; k < 4; ++k) {  // four 32-byte K slices per 128-byte row
             // K-major: the k-th 16-element slice starts 32 bytes further
             // along each 128-byte swizzled row; 8-row groups are 1024 B apart.
             const uint64_t adesc = sw128_desc(pbase + k * 32, 16, 1024);
-            // MN-major: 16 K rows of 128 B per slice; 64-element MN chunks are
-            // kBK rows apart; 8-row K groups 1024 B apart.
-            const uint64_t bdesc = Q_MN ? sw128_desc(qbase + k * 16 * 128, kBK * 128, 1024)
-                                        : sw128_desc(qbase + k * 32, 16, 1024);
-            mma_f16<1>(d, adesc, bdesc, IDESC, (!fresh || k != 0) ? 1u : 0u);
+            // MN-major: MMA_K rows of 128 B per slice; 128-byte MN chunks are
+            // KB_EL rows apart; K-row groups (8 rows; 4 rows for tf32, whose
+            // 32-byte-atom swizzle repeats every 4 rows) 1024 / 512 B apart.
+            const uint64_t bdesc =
+                Q_MN ? (TF32 ? sw128_desc(qbase + k * MMA_K * 128, KB_EL * 128, 512, 1)
+                             : sw128_desc(qbase + k * MMA_K * 128, KB_EL * 128, 1024))
+                     : sw128_desc(qbase + k * 32, 16, 1024);
+            if constexpr (TF32)
+              mma_tf32<1>(d, adesc, bdesc, IDESC, (!fresh || k != 0) ? 1u : 0u);
+            else
+              mma_f16<1>(d, adesc, bdesc, IDESC, (!fresh || k != 0) ? 1u : 0u);
           }
           mma_commit<1>(smem_u32(&empty_bar[s]));  // frees the stage when read
         }
@@ -378,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Shared memory a kernel instance needs (bytes, including alignment slack).
 template <int BN, int STAGES, bool GROUPED, bool SWAP = false>
 constexpr int gemm_smem_bytes() {
-  return 1024 + STAGES * (kBM * kBK * 2 + BN * kBK * 2) +
+  return 1024 + STAGES * (kBM * 128 + BN * 128) +
          ((!GROUPED && !SWAP) ? static_cast<int>(kEpiStageBytes) : 0) + (2 * STAGES + 5) * 8 +
          static_cast<int>(sizeof(SharedCtl)) + (GROUPED ? static_cast<int>(sizeof(GroupTable)) : 0);
 }

@@ -191,6 +191,8 @@ template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
   return __bfloat162float(v);
 }
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
 
 // Pack two fp32 values into the 32-bit pair of the output type (RNE).
 template <typename OutT>

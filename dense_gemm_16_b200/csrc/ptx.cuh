@@ -254,6 +254,26 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
         : "memory");
 }
 
+// D[tmem] (+)= A * B with fp32 operands read as tf32, one instruction (K = 8).
+template <int CG>
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+  if constexpr (CG == 1)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive (once) on `bar` when every tcgen05 op this thread issued so far has
 // completed.  `bar` is a shared::cluster address (a shared::cta address
 // names the executing CTA).
@@ -304,14 +324,27 @@ __device__ __forceinline__ void tmem_ld_wait() {
 //   lbo:   leading-dimension byte offset (MN-major: stride between 64-element
 //          MN chunks; ignored for K-major)
 //   sbo:   stride-dimension byte offset (stride between groups of 8 rows)
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t start, uint32_t lbo, uint32_t sbo) {
+//   layout: 2 = 128-byte swizzle (16-byte granules, 8-row period);
+//           1 = 128-byte swizzle with 32-byte atoms (4-row period), the only
+//               layout an MN-major 32-bit (tf32) operand may use
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t start, uint32_t lbo, uint32_t sbo,
+                                               uint32_t layout = 2) {
   uint64_t d = 0;
   d |= static_cast<uint64_t>((start >> 4) & 0x3FFFu);
   d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
   d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for tcgen05
-  d |= static_cast<uint64_t>(2) << 61;  // 128-byte swizzle
+  d |= static_cast<uint64_t>(layout & 7u) << 61;
   return d;
+}
+
+// Instruction descriptor with an fp32 accumulator for operand format `fmt`
+// (kind::f16: 0 fp16, 1 bf16; kind::tf32: 2), both operands K-major except a
+// B operand that is MN-major when b_mn = 1.
+__host__ __device__ constexpr uint32_t mma_idesc(uint32_t M, uint32_t N, uint32_t fmt,
+                                                 uint32_t b_mn) {
+  return (1u << 4) | (fmt << 7) | (fmt << 10) | (b_mn << 16) | ((N >> 3) << 17) |
+         ((M >> 4) << 24);
 }
 
 // Instruction descriptor for kind::f16 with an fp32 accumulator.

@@ -25,9 +25,10 @@
  * Memory.   Every pointer except the grouped call's host scalars is a DEVICE
  *           pointer owned by the caller.  The library never allocates,
  *           frees or keeps a reference to a caller buffer after the call.
- * Alignment. A, B and C must be 16-byte aligned; lda and ldb must be
- *           multiples of 8 elements and ldc*sizeof(output) a multiple of 16
- *           bytes (the tensor-memory-access unit copies 16-byte granules).
+ * Alignment. A, B and C must be 16-byte aligned; lda*sizeof(input),
+ *           ldb*sizeof(input) and ldc*sizeof(output) must be multiples of 16
+ *           bytes (the tensor-memory-access unit copies 16-byte granules):
+ *           multiples of 8 elements for 16-bit data, 4 for fp32.
  *           bias needs only its element alignment.  Anything else returns
  *           GEMM_ERR_MISALIGNED; there is no slower fallback.
  * Sizes.    M, N, K >= 0.  M == 0 or N == 0 is a no-op that returns GEMM_OK.
@@ -70,7 +71,10 @@ typedef enum {
   GEMM_F16 = 0,          /* fp16 in, fp32 accumulate, fp16 out (round to nearest even) */
   GEMM_BF16 = 1,         /* bf16 in, fp32 accumulate, bf16 out (round to nearest even) */
   GEMM_F16_OUT_F32 = 2,  /* fp16 in, fp32 accumulate, fp32 out */
-  GEMM_BF16_OUT_F32 = 3  /* bf16 in, fp32 accumulate, fp32 out */
+  GEMM_BF16_OUT_F32 = 3, /* bf16 in, fp32 accumulate, fp32 out */
+  GEMM_F32_TF32 = 4      /* fp32 in, multiplied as tf32 (low 13 mantissa bits ignored),
+                            fp32 accumulate, fp32 out; bias fp32; gemm() and
+                            gemm_strided_batched() only, 128 x 128/256 tiles */
 } gemm_dtype;
 
 /* `epilogue` bits. */

@@ -77,6 +77,8 @@ def _load():
             lib.oracle_decode_array.argtypes = [u16p, L, I, f64p]
             lib.oracle_gemm_f64.argtypes = [I, I, I, f64p, L, f64p, L, I, f64p, I, f64p, L, I]
             lib.oracle_gemm.argtypes = [I, I, I, u16p, L, u16p, L, I, u16p, I, I, f64p, L, I]
+            f32p = ctypes.POINTER(ctypes.c_float)
+            lib.oracle_gemm_f32.argtypes = [I, I, I, f32p, L, f32p, L, I, f32p, I, f64p, L, I]
             lib.oracle_gemm_at.argtypes = [I, I, I, u16p, L, u16p, L, I, u16p, I, I,
                                            L, i64p, i64p, f64p, I]
             lib.oracle_grouped_gemm.argtypes = [I, i32p, I, I, u16p, L, u16p, L, L, I,
@@ -169,6 +171,29 @@ def gemm(M, N, K, A, lda, B, ldb, *, b_colmajor=False, bias=None, relu=False,
     _rc(_load().oracle_gemm(M, N, K, _p(a, ctypes.c_uint16), lda, _p(b, ctypes.c_uint16), ldb,
                             int(bool(b_colmajor)), _p(bs, ctypes.c_uint16), int(bool(relu)),
                             _dt(dtype), _p(out, ctypes.c_double), max(N, 1), threads), "gemm")
+    return out
+
+
+def _f32(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().cpu().contiguous().numpy()
+    x = np.ascontiguousarray(x)
+    if x.dtype != np.float32:
+        raise TypeError("oracle: expected float32 data")
+    return x.reshape(-1)
+
+
+def gemm_f32(M, N, K, A, lda, B, ldb, *, b_colmajor=False, bias=None, relu=False,
+             threads: int = 1) -> np.ndarray:
+    """Full (M, N) float64 result from fp32 buffers addressed through lda/ldb
+    (the exact product of the fp32 values, before any tf32 rounding)."""
+    a, b, bs = _f32(A), _f32(B), _f32(bias)
+    out = np.zeros((M, N), dtype=np.float64)
+    _rc(_load().oracle_gemm_f32(M, N, K, _p(a, ctypes.c_float), lda, _p(b, ctypes.c_float), ldb,
+                                int(bool(b_colmajor)), _p(bs, ctypes.c_float), int(bool(relu)),
+                                _p(out, ctypes.c_double), max(N, 1), threads), "gemm_f32")
     return out
 
 

@@ -34,6 +34,9 @@
  *   B[k,j] = B[j*ldb + k]     if b_colmajor!=0 (column-major, stored N x K)
  *   out[i,j] = out[i*ldo + j] (double, row-major)
  *
+ * fp32 inputs (oracle_gemm_f32) follow the same definition; each value
+ * converts to double exactly.
+ *
  * Grouped variant (the MoE layer's per-expert GEMMs, "用Triton跨芯片优化GEMM"
  * section 2.3): rows of A are sorted by group; group g owns rows
  * [r_g, r_g + rows[g]) with r_g = sum_{h<g} rows[h], and uses the g-th B
@@ -191,6 +194,47 @@ int oracle_gemm(int M, int N, int K,
     if ((!K || (a && b)) && (!bias || bs))
         rc = oracle_gemm_f64(M, N, K, a, K, b, b_colmajor ? K : N, b_colmajor,
                              bs, relu, out, ldo, nthreads);
+    free(a);
+    free(b);
+    free(bs);
+    return rc;
+}
+
+/* Dense GEMM on IEEE binary32 inputs (each value is exactly representable in
+ * double, so the conversion is exact): the same definition as above.  This
+ * is what an fp32-input GEMM computes before any reduced-precision multiply
+ * (tf32) rounds its inputs. */
+int oracle_gemm_f32(int M, int N, int K,
+                    const float *A, int64_t lda,
+                    const float *B, int64_t ldb, int b_colmajor,
+                    const float *bias, int relu,
+                    double *out, int64_t ldo, int nthreads)
+{
+    if (M < 0 || N < 0 || K < 0)
+        return -1;
+    if (M == 0 || N == 0)
+        return 0;
+    if (!out || (K > 0 && (!A || !B)))
+        return -1;
+    size_t na = (size_t)M * (size_t)K;
+    size_t nb = (size_t)K * (size_t)N;
+    double *a = (double *)malloc((na ? na : 1) * sizeof(double));
+    double *b = (double *)malloc((nb ? nb : 1) * sizeof(double));
+    double *bs = bias ? (double *)malloc((size_t)N * sizeof(double)) : NULL;
+    int rc = -2;
+    if (a && b && (!bias || bs)) {
+        for (int i = 0; i < M; ++i)
+            for (int k = 0; k < K; ++k)
+                a[(size_t)i * K + k] = (double)A[(int64_t)i * lda + k];
+        /* B kept in its stored orientation */
+        int rows = b_colmajor ? N : K, cols = b_colmajor ? K : N;
+        for (int r = 0; r < rows; ++r)
+            for (int c = 0; c < cols; ++c)
+                b[(size_t)r * cols + c] = (double)B[(int64_t)r * ldb + c];
+        for (int j = 0; bias && j < N; ++j)
+            bs[j] = (double)bias[j];
+        rc = oracle_gemm_f64(M, N, K, a, K, b, cols, b_colmajor, bs, relu, out, ldo, nthreads);
+    }
     free(a);
     free(b);
     free(bs);

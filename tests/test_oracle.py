@@ -283,3 +283,38 @@ def test_tolerance_helper():
     assert ok
     ok, *_ = oracle.within_tolerance(np.array([np.nan]), np.array([1.0]), 1e-2, 1e-2)
     assert not ok
+
+
+# ------------------------------------------------------------ fp32 inputs
+
+@pytest.mark.parametrize("b_colmajor", [False, True])
+def test_f32_bruteforce_with_strides(b_colmajor):
+    rnd = random.Random(f"f32-{b_colmajor}")
+    vals = _EXACT + [3.0e-5, -7.5, 1024.125, 1.0 / 3.0]
+    for M, N, K in [(1, 1, 1), (2, 3, 4), (3, 5, 2)]:
+        A = [[np.float32(rnd.choice(vals)) for _ in range(K)] for _ in range(M)]
+        B = [[np.float32(rnd.choice(vals)) for _ in range(N)] for _ in range(K)]
+        bias = [np.float32(rnd.choice(vals)) for _ in range(N)]
+        lda, ldb = K + 3, (K + 1 if b_colmajor else N + 2)
+        a_buf = np.full(M * lda, 1e30, dtype=np.float32)
+        for i in range(M):
+            a_buf[i * lda:i * lda + K] = A[i]
+        if b_colmajor:
+            b_buf = np.full(N * ldb, -1e30, dtype=np.float32)
+            for j in range(N):
+                for k in range(K):
+                    b_buf[j * ldb + k] = B[k][j]
+        else:
+            b_buf = np.full(K * ldb, -1e30, dtype=np.float32)
+            for k in range(K):
+                b_buf[k * ldb:k * ldb + N] = B[k]
+        got = oracle.gemm_f32(M, N, K, a_buf, lda, b_buf, ldb, b_colmajor=b_colmajor,
+                              bias=np.array(bias, dtype=np.float32), relu=True)
+        # exact reference with Python fractions on the fp32 values
+        from fractions import Fraction
+        for i in range(M):
+            for j in range(N):
+                s_ = sum(Fraction(float(A[i][k])) * Fraction(float(B[k][j])) for k in range(K))
+                s_ += Fraction(float(bias[j]))
+                s_ = max(s_, Fraction(0))
+                assert abs(Fraction(got[i, j]) - s_) <= abs(s_) * Fraction(1, 2 ** 50), (i, j)

@@ -43,6 +43,8 @@ MUTANTS = {
     "bf16_exponent_off_by_one": ("ldexp((double)(128 + f), e - 134)",
                                  "ldexp((double)(128 + f), e - 133)"),
     "bf16_fraction_width": ("int f = h & 0x7f;", "int f = h & 0x3f;"),
+    "f32_lda_ignored": ("a[(size_t)i * K + k] = (double)A[(int64_t)i * lda + k];",
+                        "a[(size_t)i * K + k] = (double)A[(int64_t)i * K + k];"),
     "grouped_b_not_advanced": ("B ? B + (int64_t)g * strideB : NULL", "B"),
     "grouped_bias_not_advanced": ("bias ? bias + (int64_t)g * N : NULL,\n                                 relu",
                                   "bias,\n                                 relu"),

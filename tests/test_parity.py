@@ -420,3 +420,74 @@ def test_bmm_helper_matches_torch_layouts():
         ref = oracle.gemm(130, 72, 96, a[i].cpu(), 96, b[i].cpu(), 72, dtype="bf16",
                           threads=THREADS)
         compare(out[i].double().cpu().numpy(), ref, 2, "bmm")
+
+
+# ------------------------------------------- fp32 inputs multiplied as tf32
+
+def _tf32_bound(A, B, bias, M, N, K, b_col, ref):
+    """Error bound for fp32 inputs read as tf32: each input keeps 10 fraction
+    bits (relative error below 2^-10), so a product is off by less than
+    (2^-9 + 2^-20)|a b|; fp32 accumulation of K terms adds at most
+    K * 2^-24 * sum|a b| in any order, bias and ReLU one more rounding."""
+    S = oracle.gemm_f32(M, N, K, np.abs(A.numpy()), K, np.abs(B.numpy()), K if b_col else N,
+                        b_colmajor=b_col, bias=None if bias is None else np.abs(bias.numpy()),
+                        threads=THREADS)
+    return (2.0 ** -9 + 2.0 ** -20 + K * 2.0 ** -23) * S + 2.0 ** -22 * np.abs(ref) + 1e-30
+
+
+@pytest.mark.parametrize("config", [None, 0, 1, 8, 23])
+@pytest.mark.parametrize("b_col", [False, True])
+def test_tf32_within_its_error_bound(config, b_col):
+    M, N, K = 333, 520, 712
+    gen = torch.Generator().manual_seed(600 + (config or 0) + b_col)
+    A = torch.randn(M, K, generator=gen)
+    B = torch.randn(*((N, K) if b_col else (K, N)), generator=gen)
+    bias = torch.randn(N, generator=gen)
+    ref = oracle.gemm_f32(M, N, K, A, K, B, K if b_col else N, b_colmajor=b_col, bias=bias,
+                          relu=True, threads=THREADS)
+    if config is not None:
+        assert dg.gemm_force_config(config) == 0
+    try:
+        out = dg.matmul(A.cuda(), B.cuda(), bias=bias.cuda(), relu=True, b_col_major=b_col)
+        torch.cuda.synchronize()
+    finally:
+        dg.gemm_force_config(-1)
+    assert dg.gemm_device_status() == 0
+    got = out.double().cpu().numpy()
+    bound = _tf32_bound(A, B, bias, M, N, K, b_col, ref)
+    err = np.abs(got - ref)
+    assert np.isfinite(got).all()
+    assert (err <= bound).all(), f"max err/bound {float((err / bound).max()):.3f}"
+
+
+@pytest.mark.parametrize("b_col", [False, True])
+def test_tf32_exact_on_small_integers(b_col):
+    """Small integers are exact in tf32 and every partial sum is an integer
+    below 2^24, so the result is exact in any summation order."""
+    M, N, K = 200, 264, 600
+    gen = torch.Generator().manual_seed(77)
+    A = torch.randint(-3, 4, (M, K), generator=gen).float()
+    B = torch.randint(-3, 4, (N, K) if b_col else (K, N), generator=gen).float()
+    ref = oracle.gemm_f32(M, N, K, A, K, B, K if b_col else N, b_colmajor=b_col,
+                          threads=THREADS)
+    out = dg.matmul(A.cuda(), B.cuda(), b_col_major=b_col)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.double().cpu().numpy(), ref)
+
+
+def test_tf32_batched_and_grouped_rejection():
+    gen = torch.Generator().manual_seed(3)
+    a = torch.randn(2, 96, 64, generator=gen).cuda()
+    b = torch.randn(2, 64, 40, generator=gen).cuda()
+    out = dg.bmm(a, b)
+    torch.cuda.synchronize()
+    for i in range(2):
+        ref = oracle.gemm_f32(96, 40, 64, a[i].cpu(), 64, b[i].cpu(), 40, threads=THREADS)
+        bound = _tf32_bound(a[i].cpu(), b[i].cpu(), None, 96, 40, 64, False, ref)
+        assert (np.abs(out[i].double().cpu().numpy() - ref) <= bound).all()
+    x = torch.randn(8, 64).cuda()
+    w = torch.randn(1, 64, 16).cuda()
+    rows = torch.tensor([8], dtype=torch.int32).cuda()
+    y = torch.empty(8, 16).cuda()
+    assert dg.grouped_gemm(1, rows, 8, 16, 64, x, 64, w, 16, 1024, y, 16, None, 0,
+                           dg.GEMM_F32_TF32) == dg.GEMM_ERR_UNSUPPORTED
