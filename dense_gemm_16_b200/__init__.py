@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             L.gemm_strided_batched.argtypes = [I, I, I, I, P, L64, L64, P, L64, L64, P, L64, L64,
                                                P, L64, U, I, P]
             L.gemm_strided_batched.restype = I
+            L.conv2d_im2col.argtypes = [I] * 13 + [P, P, P, P, U, I, P]
+            L.conv2d_im2col.restype = I
             L.gemm_splitk_noalloc.argtypes = [I, I, I, P, L64, P, L64, P, L64, P, U, I, I, P]
             L.gemm_splitk_noalloc.restype = I
             _lib = L
@@ -129,6 +131,14 @@ def gemm_splitk_noalloc(M, N, K, A, lda, B, ldb, C, ldc, bias, epilogue, dtype, 
     scratch, no device allocation); returns the gemm_status."""
     return lib().gemm_splitk_noalloc(M, N, K, _ptr(A), lda, _ptr(B), ldb, _ptr(C), ldc,
                                      _ptr(bias), epilogue, dtype, splits, _stream(stream))
+
+
+def conv2d_im2col(batch, H, W, cin, cout, KH, KW, stride_h, stride_w, pad_h, pad_w, dil_h,
+                  dil_w, x, w, y, bias, epilogue, dtype, stream=None) -> int:
+    """C-ABI ``conv2d_im2col``; returns the gemm_status."""
+    return lib().conv2d_im2col(batch, H, W, cin, cout, KH, KW, stride_h, stride_w, pad_h, pad_w,
+                               dil_h, dil_w, _ptr(x), _ptr(w), _ptr(y), _ptr(bias), epilogue,
+                               dtype, _stream(stream))
 
 
 def gemm_status_string(status: int) -> str:
@@ -249,6 +259,25 @@ def bmm(a, b, bias=None, relu: bool = False, b_col_major: bool = False, out=None
     if rc:
         raise GemmError(rc, "gemm_strided_batched")
     return out
+
+
+def conv2d(x, w, bias=None, relu: bool = False, stride=(1, 1), pad=(0, 0), dil=(1, 1),
+           out_f32: bool = False, stream=None):
+    """NHWC convolution through the C ABI: x (batch, H, W, cin), w (KH, KW, cin,
+    cout) -> (batch, OH, OW, cout)."""
+    import torch
+    batch, H, W, cin = x.shape
+    KH, KW, _, cout = w.shape
+    OH = (H + 2 * pad[0] - dil[0] * (KH - 1) - 1) // stride[0] + 1
+    OW = (W + 2 * pad[1] - dil[1] * (KW - 1) - 1) // stride[1] + 1
+    y = torch.empty(batch, OH, OW, cout, device=x.device,
+                    dtype=torch.float32 if out_f32 else x.dtype)
+    epi = (GEMM_EPI_BIAS if bias is not None else 0) | (GEMM_EPI_RELU if relu else 0)
+    rc = conv2d_im2col(batch, H, W, cin, cout, KH, KW, stride[0], stride[1], pad[0], pad[1],
+                       dil[0], dil[1], x, w, y, bias, epi, dtype_code(x.dtype, out_f32), stream)
+    if rc:
+        raise GemmError(rc, "conv2d_im2col")
+    return y
 
 
 def grouped_matmul(x, w, group_rows_dev, bias=None, relu: bool = False,

@@ -3,6 +3,8 @@
 
 #include <cstdint>
 
+#include <cuda_runtime.h>
+
 namespace dg16 {
 
 // What a launch needs to know about one compiled kernel instance.
@@ -35,5 +37,10 @@ KernelEntry kernels_bn128(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_swap(int bn, bool bf16, bool out_f32);
 KernelEntry kernels_pair(int bn, int stages, bool q_mn, bool bf16, bool out_f32);
 KernelEntry kernels_tf32(int bn, bool q_mn);
+
+// NHWC im2col gather (im2col.cu): A[m][k] for M = batch*OH*OW, K = KH*KW*cin.
+cudaError_t launch_im2col(const void* x, void* A, long long lda, int batch, int H, int W, int cin,
+                          int KH, int KW, int sh, int sw, int ph, int pw, int dh, int dw, int OH,
+                          int OW, int num_sms, cudaStream_t stream);
 
 }  // namespace dg16

@@ -77,11 +77,41 @@ constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
 struct Workspace {
   int device;
   cudaStream_t stream;
+  int slot;  // 0: split/stream-K pieces (counters + partials); 1: im2col matrix
   void* ptr;
   size_t bytes;
 };
 std::mutex g_ws_mu;
 std::vector<Workspace> g_ws;
+
+// Plain per-(device, stream, slot) scratch of at least `bytes` (slot 1 and
+// up; contents undefined).  Same growth rule as stream_workspace.
+int stream_buffer(int device, cudaStream_t stream, int slot, size_t bytes, void** out) {
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  Workspace* w = nullptr;
+  for (auto& e : g_ws)
+    if (e.device == device && e.stream == stream && e.slot == slot) w = &e;
+  if (!w || w->bytes < bytes) {
+    if (w) {
+      cudaError_t e = cudaStreamSynchronize(stream);
+      if (e != cudaSuccess) return cuda_fail(e);
+      cudaFree(w->ptr);
+      w->ptr = nullptr;
+      w->bytes = 0;
+    } else {
+      g_ws.push_back({device, stream, slot, nullptr, 0});
+      w = &g_ws.back();
+    }
+    const size_t sz = std::max(bytes, static_cast<size_t>(16) << 20);
+    void* ptr = nullptr;
+    cudaError_t e = cudaMalloc(&ptr, sz);
+    if (e != cudaSuccess) return cuda_fail(e);
+    w->ptr = ptr;
+    w->bytes = sz;
+  }
+  *out = w->ptr;
+  return GEMM_OK;
+}
 
 // Scratch of at least `partial_bytes` after the counters for (device, stream).
 // The first call per stream allocates (cudaMalloc) and zeroes the counters;
@@ -93,7 +123,7 @@ int stream_workspace(int device, cudaStream_t stream, size_t partial_bytes, floa
   const size_t need = kCounterBytes + partial_bytes;
   Workspace* w = nullptr;
   for (auto& e : g_ws)
-    if (e.device == device && e.stream == stream) w = &e;
+    if (e.device == device && e.stream == stream && e.slot == 0) w = &e;
   if (!w || w->bytes < need) {
     if (w) {
       cudaError_t e = cudaStreamSynchronize(stream);
@@ -102,7 +132,7 @@ int stream_workspace(int device, cudaStream_t stream, size_t partial_bytes, floa
       w->ptr = nullptr;
       w->bytes = 0;
     } else {
-      g_ws.push_back({device, stream, nullptr, 0});
+      g_ws.push_back({device, stream, 0, nullptr, 0});
       w = &g_ws.back();
     }
     const size_t bytes = std::max(need, static_cast<size_t>(16) << 20);
@@ -604,6 +634,49 @@ int gemm_strided_batched(int batch, int M, int N, int K, const void* A, int64_t 
     const long long tiles256 = static_cast<long long>((M + 127) / 128) * ((N + 255) / 256);
     cid = (N <= 128 || tiles256 < 96) ? 1 : 0;
   }
+  return run_dense(ds, d, kConfigs[cid], kConfigs[cid].splits, nullptr, stream);
+}
+
+int conv2d_im2col(int batch, int H, int W, int cin, int cout, int KH, int KW, int stride_h,
+                  int stride_w, int pad_h, int pad_w, int dil_h, int dil_w, const void* x,
+                  const void* w, void* y, const void* bias, unsigned epilogue, int dtype,
+                  void* stream_) {
+  int rc = check_dtype_epi(epilogue, dtype);
+  if (rc) return rc;
+  if (epilogue & GEMM_B_COL_MAJOR) return GEMM_ERR_UNSUPPORTED;  // the filter layout is fixed
+  if (in_tf32(dtype)) return GEMM_ERR_UNSUPPORTED;               // 16-bit activations only
+  if (batch < 0 || H < 1 || W < 1 || cin < 1 || cout < 1 || KH < 1 || KW < 1 || stride_h < 1 ||
+      stride_w < 1 || pad_h < 0 || pad_w < 0 || dil_h < 1 || dil_w < 1)
+    return GEMM_ERR_INVALID_ARG;
+  const int OH = (H + 2 * pad_h - dil_h * (KH - 1) - 1) / stride_h + 1;
+  const int OW = (W + 2 * pad_w - dil_w * (KW - 1) - 1) / stride_w + 1;
+  if (OH < 1 || OW < 1) return GEMM_ERR_INVALID_ARG;
+  if (batch == 0) return GEMM_OK;
+  if (!x || !w || !y || ((epilogue & GEMM_EPI_BIAS) && !bias)) return GEMM_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y) ||
+      (static_cast<int64_t>(cout) * out_bytes(dtype)) % 16 != 0 || cout % 8 != 0)
+    return GEMM_ERR_MISALIGNED;
+  const long long M = static_cast<long long>(batch) * OH * OW;
+  const long long K = static_cast<long long>(KH) * KW * cin;
+  if (M > INT32_MAX || K > INT32_MAX) return GEMM_ERR_UNSUPPORTED;
+  const long long lda = (K + 7) / 8 * 8;  // 16-byte rows for the TMA
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  DeviceState* ds = nullptr;
+  rc = device_state(&ds);
+  if (rc) return rc;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  void* A = nullptr;
+  rc = stream_buffer(dev, stream, 1, static_cast<size_t>(M) * lda * 2, &A);
+  if (rc) return rc;
+  e = launch_im2col(x, A, lda, batch, H, W, cin, KH, KW, stride_h, stride_w, pad_h, pad_w, dil_h,
+                    dil_w, OH, OW, ds->num_sms, stream);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const DenseProblem d{1,     static_cast<int>(M), cout, static_cast<int>(K), A, lda, 0, w, cout,
+                       0,     y, cout, 0, bias, 0, epilogue, dtype};
+  const int cid = select_config(d.M, d.N, d.K, epilogue, false);
+  if (cid < 0 || cid >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
   return run_dense(ds, d, kConfigs[cid], kConfigs[cid].splits, nullptr, stream);
 }
 

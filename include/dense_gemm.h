@@ -23,8 +23,13 @@
  *             C[i,j] = C[i*ldc + j]                        (row-major, M x N)
  *           bias is a length-N vector of the input type, broadcast over rows.
  * Memory.   Every pointer except the grouped call's host scalars is a DEVICE
- *           pointer owned by the caller.  The library never allocates,
- *           frees or keeps a reference to a caller buffer after the call.
+ *           pointer owned by the caller.  The library never frees or keeps
+ *           a reference to a caller buffer after the call.  Its own device
+ *           memory is a status word per device and, only for calls that need
+ *           it, per-stream scratch: split-K / stream-K partial tiles and the
+ *           im2col matrix of conv2d_im2col, each allocated with cudaMalloc on
+ *           the first such call on a stream and grown on demand
+ *           (gemm_splitk_noalloc never allocates).
  * Alignment. A, B and C must be 16-byte aligned; lda*sizeof(input),
  *           ldb*sizeof(input) and ldc*sizeof(output) must be multiples of 16
  *           bytes (the tensor-memory-access unit copies 16-byte granules):
@@ -130,6 +135,32 @@ GEMM_API int gemm_strided_batched(int batch, int M, int N, int K, const void* A,
                                   int64_t stride_a, const void* B, int64_t ldb, int64_t stride_b,
                                   void* C, int64_t ldc, int64_t stride_c, const void* bias,
                                   int64_t stride_bias, unsigned epilogue, int dtype, void* stream);
+
+/*
+ * conv2d_im2col -- 2-D convolution as a GEMM ("FlagOS众智跨芯算子优化实践"
+ * section 5.3: convolution reuses the GEMM through im2col):
+ *
+ *   y[n][oh][ow][co] = act( sum_{kh,kw,ci} x[n][ih][iw][ci] * w[kh][kw][ci][co] + bias[co] )
+ *   ih = oh*stride_h - pad_h + kh*dil_h,  iw = ow*stride_w - pad_w + kw*dil_w,
+ *
+ * x taken as 0 outside the image.  The sliding windows are gathered into an
+ * (batch*OH*OW) x (KH*KW*cin) matrix, then multiplied by the filter on the
+ * tensor cores with bias and ReLU fused into the GEMM epilogue.
+ *
+ *   x      device, NHWC [batch][H][W][cin], 16-bit (dtype GEMM_F16/BF16[_OUT_F32])
+ *   w      device, [KH][KW][cin][cout] (a K x N row-major matrix, K = KH*KW*cin)
+ *   y      device, NHWC [batch][OH][OW][cout], OH = (H + 2 pad_h - dil_h (KH-1) - 1)
+ *          / stride_h + 1, OW likewise
+ *   bias   device, cout elements iff GEMM_EPI_BIAS
+ *   epilogue  GEMM_EPI_BIAS | GEMM_EPI_RELU (no layout bits)
+ * cout must be a multiple of 8; x, w, y 16-byte aligned.  The gathered matrix
+ * lives in a per-stream scratch buffer the library allocates (cudaMalloc) on
+ * the first call on a stream and grows when a larger one is needed.
+ */
+GEMM_API int conv2d_im2col(int batch, int H, int W, int cin, int cout, int KH, int KW,
+                           int stride_h, int stride_w, int pad_h, int pad_w, int dil_h, int dil_w,
+                           const void* x, const void* w, void* y, const void* bias,
+                           unsigned epilogue, int dtype, void* stream);
 
 /*
  * grouped_gemm -- the per-expert GEMMs of an MoE layer in one launch

@@ -86,6 +86,7 @@ def _load():
             lib.oracle_grouped_gemm_at.argtypes = [I, i32p, I, I, u16p, L, u16p, L, L, I,
                                                    u16p, I, I, L, i64p, i64p, f64p, I]
             lib.oracle_threads_used.argtypes = [I]
+            lib.oracle_conv2d_nhwc.argtypes = [I] * 13 + [u16p, u16p, u16p, I, I, f64p, I]
             _lib = lib
     return _lib
 
@@ -266,3 +267,29 @@ def within_tolerance(got: np.ndarray, ref: np.ndarray, atol: float, rtol: float)
     worst = int(np.argmax(excess))
     rel = err / np.maximum(np.abs(ref), 1e-30)
     return ok, float(np.nanmax(err)), float(np.nanmax(np.where(np.abs(ref) > 0, rel, 0.0))), worst
+
+
+def conv_out_size(H, W, KH, KW, stride=(1, 1), pad=(0, 0), dil=(1, 1)):
+    OH = (H + 2 * pad[0] - dil[0] * (KH - 1) - 1) // stride[0] + 1
+    OW = (W + 2 * pad[1] - dil[1] * (KW - 1) - 1) // stride[1] + 1
+    return OH, OW
+
+
+def conv2d_nhwc(x, w, *, stride=(1, 1), pad=(0, 0), dil=(1, 1), bias=None, relu=False,
+                dtype="f16", threads: int = 1) -> np.ndarray:
+    """Direct NHWC convolution: x (batch, H, W, cin), w (KH, KW, cin, cout)
+    -> (batch, OH, OW, cout) float64."""
+    batch, H, W, cin = x.shape
+    KH, KW, cin2, cout = w.shape
+    if cin2 != cin:
+        raise ValueError("oracle: channel counts differ")
+    OH, OW = conv_out_size(H, W, KH, KW, stride, pad, dil)
+    xb, wb = _bits(x), _bits(w)
+    bs = None if bias is None else _bits(bias)
+    out = np.zeros((batch, OH, OW, cout), dtype=np.float64)
+    _rc(_load().oracle_conv2d_nhwc(batch, H, W, cin, cout, KH, KW, stride[0], stride[1], pad[0],
+                                   pad[1], dil[0], dil[1], _p(xb, ctypes.c_uint16),
+                                   _p(wb, ctypes.c_uint16), _p(bs, ctypes.c_uint16),
+                                   int(bool(relu)), _dt(dtype), _p(out, ctypes.c_double),
+                                   threads), "conv2d_nhwc")
+    return out

@@ -288,6 +288,67 @@ int oracle_gemm_at(int M, int N, int K,
     return 0;
 }
 
+/* 2-D convolution, NHWC activations, straight from its definition ("FlagOS
+ * 众智跨芯算子优化实践" section 5.3 names convolution as the first operator
+ * to reuse the GEMM: it is the same sum of products over a sliding window):
+ *
+ *   y[n][oh][ow][co] = act( sum_{kh,kw,ci} x[n][ih][iw][ci] * w[kh][kw][ci][co]
+ *                           + bias[co] ),  ih = oh*sh - ph + kh*dh,
+ *                                          iw = ow*sw - pw + kw*dw,
+ *
+ * with x taken as 0 outside [0,H) x [0,W) (zero padding).  x is
+ * [batch][H][W][cin], w is [KH][KW][cin][cout], y is [batch][OH][OW][cout]
+ * (double), OH = (H + 2ph - dh(KH-1) - 1)/sh + 1, OW likewise.  The sum runs
+ * kh, kw, ci ascending in fp64. */
+int oracle_conv2d_nhwc(int batch, int H, int W, int cin, int cout, int KH, int KW,
+                       int sh, int sw, int ph, int pw, int dh, int dw,
+                       const uint16_t *x, const uint16_t *w, const uint16_t *bias,
+                       int relu, int dtype, double *y, int nthreads)
+{
+    if (batch < 0 || H < 1 || W < 1 || cin < 1 || cout < 1 || KH < 1 || KW < 1 ||
+        sh < 1 || sw < 1 || ph < 0 || pw < 0 || dh < 1 || dw < 1 ||
+        (dtype != ORACLE_F16 && dtype != ORACLE_BF16))
+        return -1;
+    const int OH = (H + 2 * ph - dh * (KH - 1) - 1) / sh + 1;
+    const int OW = (W + 2 * pw - dw * (KW - 1) - 1) / sw + 1;
+    if (OH < 1 || OW < 1)
+        return -1;
+    if (!x || !w || !y)
+        return -1;
+    if (nthreads < 1)
+        nthreads = 1;
+    (void)nthreads;
+    const int64_t rows = (int64_t)batch * OH * OW;
+#pragma omp parallel for num_threads(nthreads) schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const int n = (int)(r / ((int64_t)OH * OW));
+        const int oh = (int)((r / OW) % OH);
+        const int ow = (int)(r % OW);
+        for (int co = 0; co < cout; ++co) {
+            double s = 0.0;
+            for (int kh = 0; kh < KH; ++kh) {
+                const int ih = oh * sh - ph + kh * dh;
+                for (int kw = 0; kw < KW; ++kw) {
+                    const int iw = ow * sw - pw + kw * dw;
+                    if (ih < 0 || ih >= H || iw < 0 || iw >= W)
+                        continue;  /* zero padding contributes nothing */
+                    for (int ci = 0; ci < cin; ++ci) {
+                        double a = decode(x[(((int64_t)n * H + ih) * W + iw) * cin + ci], dtype);
+                        double b = decode(w[(((int64_t)kh * KW + kw) * cin + ci) * cout + co], dtype);
+                        s += a * b;
+                    }
+                }
+            }
+            if (bias)
+                s += decode(bias[co], dtype);
+            if (relu && s < 0.0)
+                s = 0.0;
+            y[r * cout + co] = s;
+        }
+    }
+    return 0;
+}
+
 /* Group that owns global row r, and that group's first row; -1 if none. */
 static int group_of_row(int G, const int32_t *group_rows, int64_t r,
                         int64_t *first)

@@ -185,3 +185,19 @@ def test_batched_argument_errors(args, expect):
 def test_batched_empty_is_a_noop():
     assert dg.lib().gemm_strided_batched(0, 4, 4, 4, P, 8, 32, P, 8, 32, P, 8, 32, None, 0, 0, 0,
                                          None) == 0
+
+
+@pytest.mark.parametrize("args,expect", [
+    # (batch, H, W, cin, cout, KH, KW, sh, sw, ph, pw, dh, dw, x, w, y, bias, epi, dtype)
+    ((1, 8, 8, 4, 8, 3, 3, 1, 1, 1, 1, 1, 1, P, P, P, None, 0, 9), dg.GEMM_ERR_UNSUPPORTED),
+    ((1, 8, 8, 4, 8, 3, 3, 1, 1, 1, 1, 1, 1, P, P, P, None, 0x100, 0), dg.GEMM_ERR_UNSUPPORTED),
+    ((1, 8, 8, 4, 8, 3, 3, 0, 1, 1, 1, 1, 1, P, P, P, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),
+    ((1, 2, 2, 4, 8, 5, 5, 1, 1, 0, 0, 1, 1, P, P, P, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),
+    ((1, 8, 8, 4, 8, 3, 3, 1, 1, 1, 1, 1, 1, None, P, P, None, 0, 0), dg.GEMM_ERR_INVALID_ARG),
+    ((1, 8, 8, 4, 8, 3, 3, 1, 1, 1, 1, 1, 1, P, P, P, None, 1, 0), dg.GEMM_ERR_INVALID_ARG),
+    ((1, 8, 8, 4, 12, 3, 3, 1, 1, 1, 1, 1, 1, P, P, P, None, 0, 0), dg.GEMM_ERR_MISALIGNED),
+    ((1, 8, 8, 4, 8, 3, 3, 1, 1, 1, 1, 1, 1, P + 2, P, P, None, 0, 0), dg.GEMM_ERR_MISALIGNED),
+    ((1, 8, 8, 4, 8, 3, 3, 1, 1, 1, 1, 1, 1, P, P, P, None, 0, 4), dg.GEMM_ERR_UNSUPPORTED),
+])
+def test_conv_argument_errors(args, expect):
+    assert dg.lib().conv2d_im2col(*args, None) == expect

@@ -318,3 +318,66 @@ def test_f32_bruteforce_with_strides(b_colmajor):
                 s_ += Fraction(float(bias[j]))
                 s_ = max(s_, Fraction(0))
                 assert abs(Fraction(got[i, j]) - s_) <= abs(s_) * Fraction(1, 2 ** 50), (i, j)
+
+
+# ------------------------------------------------------------ convolution
+
+def _conv_brute(x, w, stride, pad, dil, bias, relu):
+    """Direct convolution on nested Python lists of exact floats."""
+    batch, H, W, cin = len(x), len(x[0]), len(x[0][0]), len(x[0][0][0])
+    KH, KW, cout = len(w), len(w[0]), len(w[0][0][0])
+    OH, OW = oracle.conv_out_size(H, W, KH, KW, stride, pad, dil)
+    y = [[[[0.0] * cout for _ in range(OW)] for _ in range(OH)] for _ in range(batch)]
+    for n in range(batch):
+        for oh in range(OH):
+            for ow in range(OW):
+                for co in range(cout):
+                    s_ = 0.0
+                    for kh in range(KH):
+                        for kw in range(KW):
+                            ih = oh * stride[0] - pad[0] + kh * dil[0]
+                            iw = ow * stride[1] - pad[1] + kw * dil[1]
+                            if 0 <= ih < H and 0 <= iw < W:
+                                for ci in range(cin):
+                                    s_ += x[n][ih][iw][ci] * w[kh][kw][ci][co]
+                    if bias is not None:
+                        s_ += bias[co]
+                    y[n][oh][ow][co] = max(s_, 0.0) if relu else s_
+    return y
+
+
+@pytest.mark.parametrize("geom", [((1, 1), (0, 0), (1, 1)), ((1, 1), (1, 1), (1, 1)),
+                                  ((2, 1), (1, 2), (1, 1)), ((1, 2), (2, 1), (2, 1))])
+def test_conv_bruteforce(geom):
+    stride, pad, dil = geom
+    rnd = random.Random(str(geom))
+    batch, H, W, cin, cout, KH, KW = 2, 5, 4, 3, 2, 3, 2
+    x = [[[[rnd.choice(_EXACT) for _ in range(cin)] for _ in range(W)] for _ in range(H)]
+         for _ in range(batch)]
+    w = [[[[rnd.choice(_EXACT) for _ in range(cout)] for _ in range(cin)] for _ in range(KW)]
+         for _ in range(KH)]
+    bias = [rnd.choice(_EXACT) for _ in range(cout)]
+    xt = torch.tensor(x, dtype=torch.float64).half()
+    wt = torch.tensor(w, dtype=torch.float64).half()
+    got = oracle.conv2d_nhwc(xt, wt, stride=stride, pad=pad, dil=dil,
+                             bias=torch.tensor(bias).half(), relu=True)
+    assert np.array_equal(got, np.array(_conv_brute(x, w, stride, pad, dil, bias, True)))
+
+
+def test_conv_delta_filter_copies_the_input():
+    x = _rand_bits((2, 6, 7, 4), "bf16", 21)
+    w = torch.zeros(3, 3, 4, 4, dtype=torch.bfloat16)
+    for c in range(4):
+        w[1, 1, c, c] = 1  # centre tap, channel c -> c
+    got = oracle.conv2d_nhwc(x, w, pad=(1, 1), dtype="bf16")
+    assert np.array_equal(got, x.double().numpy())
+
+
+def test_conv_1x1_is_a_matrix_product():
+    x = _rand_bits((2, 3, 5, 8), "f16", 22)
+    w = _rand_bits((1, 1, 8, 6), "f16", 23)
+    got = oracle.conv2d_nhwc(x, w)
+    xs = x.double().numpy().reshape(-1, 8)
+    ws = w.double().numpy().reshape(8, 6)
+    exp = [[sum(xs[r, k] * ws[k, c] for k in range(8)) for c in range(6)] for r in range(xs.shape[0])]
+    assert np.allclose(got.reshape(-1, 6), np.array(exp), rtol=0, atol=1e-12)

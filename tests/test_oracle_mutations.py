@@ -45,6 +45,10 @@ MUTANTS = {
     "bf16_fraction_width": ("int f = h & 0x7f;", "int f = h & 0x3f;"),
     "f32_lda_ignored": ("a[(size_t)i * K + k] = (double)A[(int64_t)i * lda + k];",
                         "a[(size_t)i * K + k] = (double)A[(int64_t)i * K + k];"),
+    "conv_pad_sign": ("const int ih = oh * sh - ph + kh * dh;",
+                      "const int ih = oh * sh + ph + kh * dh;"),
+    "conv_dilation_ignored": ("const int iw = ow * sw - pw + kw * dw;",
+                              "const int iw = ow * sw - pw + kw;"),
     "grouped_b_not_advanced": ("B ? B + (int64_t)g * strideB : NULL", "B"),
     "grouped_bias_not_advanced": ("bias ? bias + (int64_t)g * N : NULL,\n                                 relu",
                                   "bias,\n                                 relu"),

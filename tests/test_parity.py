@@ -491,3 +491,30 @@ def test_tf32_batched_and_grouped_rejection():
     y = torch.empty(8, 16).cuda()
     assert dg.grouped_gemm(1, rows, 8, 16, 64, x, 64, w, 16, 1024, y, 16, None, 0,
                            dg.GEMM_F32_TF32) == dg.GEMM_ERR_UNSUPPORTED
+
+
+# ------------------------------------------------------ im2col convolution
+
+@pytest.mark.parametrize("shape", [
+    # batch, H, W, cin, cout, KH, KW, stride, pad, dil
+    (2, 14, 14, 64, 128, 3, 3, (1, 1), (1, 1), (1, 1)),    # 3x3 same-padding
+    (1, 17, 23, 32, 64, 3, 3, (2, 2), (1, 1), (1, 1)),     # stride 2, ragged image
+    (2, 12, 12, 16, 40, 3, 3, (1, 1), (2, 2), (2, 2)),     # dilated
+    (3, 9, 10, 64, 96, 1, 1, (1, 1), (0, 0), (1, 1)),      # 1x1 (a plain GEMM)
+    (2, 20, 18, 3, 16, 5, 5, (1, 2), (2, 1), (1, 1)),      # 3 input channels (scalar gather)
+])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_conv2d_im2col(shape, dtype):
+    batch, H, W, cin, cout, KH, KW, stride, pad, dil = shape
+    gen = torch.Generator().manual_seed(sum(shape[:7]))
+    x = (torch.rand(batch, H, W, cin, generator=gen) * 2 - 1).to(dtype)
+    w = (torch.randn(KH, KW, cin, cout, generator=gen) * 0.2).to(dtype)
+    bias = torch.randn(cout, generator=gen).to(dtype)
+    y = dg.conv2d(x.cuda(), w.cuda(), bias=bias.cuda(), relu=True, stride=stride, pad=pad,
+                  dil=dil)
+    torch.cuda.synchronize()
+    assert dg.gemm_device_status() == 0
+    ref = oracle.conv2d_nhwc(x, w, stride=stride, pad=pad, dil=dil, bias=bias, relu=True,
+                             dtype="bf16" if dtype == torch.bfloat16 else "f16",
+                             threads=THREADS)
+    compare(y.double().cpu().numpy(), ref, 2, f"conv {shape}")
