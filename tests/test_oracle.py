@@ -347,7 +347,8 @@ def _conv_brute(x, w, stride, pad, dil, bias, relu):
 
 
 @pytest.mark.parametrize("geom", [((1, 1), (0, 0), (1, 1)), ((1, 1), (1, 1), (1, 1)),
-                                  ((2, 1), (1, 2), (1, 1)), ((1, 2), (2, 1), (2, 1))])
+                                  ((2, 1), (1, 2), (1, 1)), ((1, 2), (2, 1), (2, 1)),
+                                  ((1, 1), (0, 1), (2, 2))])
 def test_conv_bruteforce(geom):
     stride, pad, dil = geom
     rnd = random.Random(str(geom))
