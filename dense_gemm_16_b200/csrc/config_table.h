@@ -41,6 +41,9 @@ static const Config kConfigs[] = {
     {"swap_128x32_s8_sk", kKindSwap, 32, 8, 1, -1, 1, 2},
     {"tc1_128x128_s6_g8_sk", kKindSingle, 128, 6, 8, -1, 2, 2},
     {"tc1_128x256_s4_g8_sk", kKindSingle, 256, 4, 8, -1, 2, 2},
+    {"gswap_128x256_s4", kKindGroupedSwap, 256, 4, 1, 1, 0, 0},
+    {"gswap2_256x256_s6", kKindGroupedSwapPair, 256, 6, 1, 1, 0, 0},
+    {"gswap2_256x256_s6_xl", kKindGroupedSwapPair, 256, 6, 1, 1, 0, 2},
 };
 static constexpr int kNumConfigs = static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0]));
 
@@ -63,7 +66,9 @@ static const Rule kRules[] = {
     {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 16},  // m1000n1000k2000_bcol: tc1_128x128_s6_g8_pn 186 TFLOP/s
     {4096, 4096, 4096, 4096, 512, 512, 1, 0, 1},  // m4096n4096k512_bcol: tc1_128x128_s6_g8 509 TFLOP/s
     {16, 16, 8192, 8192, 8192, 8192, 1, 0, 6},  // m16n8192k8192_bcol: swap_128x16_s8_k4 61 TFLOP/s
-    {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 716 TFLOP/s (grouped ignores split-K)
+    {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 704 TFLOP/s
+    {16384, 16384, 4096, 4096, 4096, 4096, 0, 1, 0},  // moe8_n4096_k4096: tc1_128x256_s4_g8 1228 TFLOP/s
+    {8192, 8192, 768, 768, 2048, 2048, 0, 1, 27},  // moe64_n768_k2048: gswap2_256x256_s6_xl 331 TFLOP/s
     {0, 0, 0, 0, 0, 0, -1, -1, -1},  // sentinel
 };
 // END RULES

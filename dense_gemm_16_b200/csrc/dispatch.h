@@ -17,6 +17,9 @@ enum ConfigKind : int {
   kKindSingle = 0,  // one CTA per 128 x BN tile
   kKindSwap = 1,    // skinny problems: C^T = B^T A^T, N fills the MMA rows
   kKindPair = 2,    // two CTAs (cta_group::2) per 256 x BN tile
+  kKindGroupedSwap = 3,  // grouped only: Y_g^T tiles of 128 columns x <= bn rows,
+                         // sized per group, drawn from a dynamic tile queue
+  kKindGroupedSwapPair = 4,  // the same with a CTA pair per 256 columns x <= bn rows
 };
 
 struct Config {
@@ -37,6 +40,8 @@ KernelEntry kernels_bn128(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_swap(int bn, bool bf16, bool out_f32);
 KernelEntry kernels_pair(int bn, int stages, bool q_mn, bool bf16, bool out_f32);
 KernelEntry kernels_tf32(int bn, bool q_mn);
+KernelEntry kernels_gswap(int tok, bool p_mn, bool bf16, bool out_f32);
+KernelEntry kernels_gswap2(int tok, bool p_mn, bool bf16, bool out_f32);
 
 // NHWC im2col gather (im2col.cu): A[m][k] for M = batch*OH*OW, K = KH*KW*cin.
 cudaError_t launch_im2col(const void* x, void* A, long long lda, int batch, int H, int W, int cin,

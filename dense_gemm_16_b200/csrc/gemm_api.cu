@@ -18,6 +18,7 @@
 #include "config_table.h"
 #include "dispatch.h"
 #include "gemm_kernel.cuh"
+#include "gemm_kernel_gswap.cuh"
 #include "raster.h"
 
 namespace dg16 {
@@ -71,9 +72,12 @@ int cuda_fail(cudaError_t e) {
 
 // Split-K scratch, one buffer per (device, stream): calls on one stream run
 // in order, so they can share it; calls on different streams never do.
-// Layout: [kCounterSlots unsigned counters, zeroed once][partial tiles].
+// Layout: [kCounterSlots tile counters][kSchedSlots tile-queue counters]
+// [partial tiles]; the counters are zeroed once and every kernel leaves
+// them at 0.
 constexpr size_t kCounterSlots = 65536;
-constexpr size_t kCounterBytes = kCounterSlots * sizeof(unsigned);
+constexpr size_t kSchedSlots = 64;  // slot 0: the grouped-swap tile queue
+constexpr size_t kCounterBytes = (kCounterSlots + kSchedSlots) * sizeof(unsigned);
 struct Workspace {
   int device;
   cudaStream_t stream;
@@ -302,6 +306,11 @@ KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool gro
   if (c.kind == kKindSwap) {
     if (q_mn || grouped) return {nullptr, 0};  // needs column-major B
     return kernels_swap(c.bn, bf16, f32);
+  }
+  if (c.kind == kKindGroupedSwap || c.kind == kKindGroupedSwapPair) {
+    if (!grouped) return {nullptr, 0};
+    return c.kind == kKindGroupedSwap ? kernels_gswap(c.bn, q_mn, bf16, f32)
+                                      : kernels_gswap2(c.bn, q_mn, bf16, f32);
   }
   if (c.kind == kKindPair) {
     if (grouped) return {nullptr, 0};
@@ -680,6 +689,91 @@ int conv2d_im2col(int batch, int H, int W, int cin, int cout, int KH, int KW, in
   return run_dense(ds, d, kConfigs[cid], kConfigs[cid].splits, nullptr, stream);
 }
 
+// Grouped GEMM with swapped operands (gemm_gswap_kernel, or the CTA-pair
+// gemm_gswap2_kernel): W_g is the 128-row (pair: 256-row) MMA operand, X's
+// rows the MMA's N; tiles come from a counter in the stream's scratch, which
+// every launch leaves at 0.
+int launch_grouped_swap(DeviceState* ds, const KernelEntry& k, const Config& cfg, int num_groups,
+                        const int32_t* group_rows, int total_rows, int N, int K, const void* A,
+                        int64_t lda, const void* B, int64_t ldb, int64_t stride_b, void* C,
+                        int64_t ldc, const void* bias, unsigned epilogue, bool bf16,
+                        cudaStream_t stream) {
+  const bool bcol = (epilogue & GEMM_B_COL_MAJOR) != 0;
+  CUtensorMap tw;
+  const uint64_t sW[2] = {static_cast<uint64_t>(ldb) * 2,
+                          num_groups > 1 ? static_cast<uint64_t>(stride_b) * 2
+                                         : static_cast<uint64_t>(bcol ? N : K) * ldb * 2};
+  int rc;
+  if (bcol) {  // W_g stored N x K: K-major boxes of 64 K x 128 columns
+    const uint64_t d[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N),
+                           static_cast<uint64_t>(num_groups)};
+    const uint32_t b[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM), 1u};
+    rc = make_map(&tw, B, bf16, 3, d, sW, b);
+  } else {  // W_g stored K x N: MN-major boxes of 64 columns x 64 K
+    const uint64_t d[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K),
+                           static_cast<uint64_t>(num_groups)};
+    const uint32_t b[3] = {64u, static_cast<uint32_t>(kBK), 1u};
+    rc = make_map(&tw, B, bf16, 3, d, sW, b);
+  }
+  if (rc) return rc;
+  RowMaps tx;
+  const uint64_t dX[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(total_rows)};
+  const uint64_t sX = static_cast<uint64_t>(lda) * 2;
+  for (int i = 0; i < 5; ++i) {
+    const uint32_t b[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(128 >> i)};
+    rc = make_map(&tx.m[i], A, bf16, 2, dX, &sX, b);
+    if (rc) return rc;
+  }
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  float* ws = nullptr;
+  unsigned* counters = nullptr;
+  rc = stream_workspace(dev, stream, 0, &ws, &counters);
+  if (rc) return rc;
+
+  KParams kp = {};
+  kp.M = total_rows;
+  kp.N = N;
+  kp.K = K;
+  kp.num_kb = (K + kBK - 1) / kBK;
+  kp.group_m = 1;
+  kp.C = C;
+  kp.ldc = ldc;
+  kp.bias = bias;
+  kp.epi = static_cast<int>(epilogue & 3);
+  kp.group_rows = group_rows;
+  kp.num_groups = num_groups;
+  kp.status = ds->status;
+  kp.timeout_ns = g_timeout_ns.load();
+  kp.pol_p = cfg.pol_p;
+  kp.pol_q = cfg.pol_q;
+  kp.counters = counters + kCounterSlots;  // the tile-queue counter
+  const bool pair = cfg.kind == kKindGroupedSwapPair;
+  const long long cols = pair ? 2 * kBM : kBM;
+  const long long nb = (N + cols - 1) / cols;
+  const long long max_tiles = (static_cast<long long>(total_rows) / cfg.bn + num_groups) * nb;
+  const int grid = pair ? 2 * static_cast<int>(std::min<long long>(max_tiles, ds->num_sms / 2))
+                        : static_cast<int>(std::min<long long>(max_tiles, ds->num_sms));
+  cudaLaunchConfig_t lc = {};
+  cudaLaunchAttribute attr[1];
+  lc.gridDim = dim3(grid, 1, 1);
+  lc.blockDim = dim3(kThreads, 1, 1);
+  lc.dynamicSmemBytes = k.smem;
+  lc.stream = stream;
+  if (pair) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    lc.attrs = attr;
+    lc.numAttrs = 1;
+  }
+  void* args[3] = {&tw, &tx, &kp};
+  e = cudaLaunchKernelExC(&lc, k.fn, args);
+  return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
+}
+
 int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int N, int K,
                  const void* A, int64_t lda, const void* B, int64_t ldb, int64_t stride_b,
                  void* C, int64_t ldc, const void* bias, unsigned epilogue, int dtype,
@@ -729,6 +823,9 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
   if (!k.fn) return GEMM_ERR_UNSUPPORTED;
   rc = ensure_smem_attr(ds, k);
   if (rc) return rc;
+  if (cfg.kind == kKindGroupedSwap || cfg.kind == kKindGroupedSwapPair)
+    return launch_grouped_swap(ds, k, cfg, num_groups, group_rows, total_rows, N, K, A, lda, B,
+                               ldb, stride_b, C, ldc, bias, epilogue, bf16, stream);
 
   CUtensorMap tp, tq;
   const uint64_t lda_b = static_cast<uint64_t>(lda) * 2;

@@ -103,6 +103,8 @@ def _dense_calls(dg, torch, names, M, N, K, dtype, b_col):
     for cid, name in enumerate(names):
         if name.startswith("swap") and not b_col:
             skipped[cid] = "needs column-major B"
+        elif name.startswith("gswap"):
+            skipped[cid] = "grouped only"
         else:
             calls[cid] = make()
     return calls, skipped, keep
@@ -112,6 +114,8 @@ def _dense_calls(dg, torch, names, M, N, K, dtype, b_col):
 # Dirichlet/multinomial routing of the MoE workload.
 GROUPED_CLASSES = [
     ("moe32_n1408_k4096", 32, 8192, 1408, 4096, "bf16"),
+    ("moe8_n4096_k4096", 8, 16384, 4096, 4096, "bf16"),
+    ("moe64_n768_k2048", 64, 8192, 768, 2048, "bf16"),
 ]
 
 
@@ -134,8 +138,8 @@ def _grouped_calls(dg, torch, names, E, R, N, K, dtype):
                                 dg.GEMM_EPI_RELU, code, stream)
     calls, skipped = {}, {}
     for cid, name in enumerate(names):
-        if name.startswith(("swap", "pair")) or "_k" in name:
-            skipped[cid] = "not a grouped kernel (or split-K, which grouped ignores)"
+        if name.startswith(("swap", "pair")) or "_k" in name or name.endswith("_sk"):
+            skipped[cid] = "not a grouped kernel (or split-K / stream-K, which grouped ignores)"
         else:
             calls[cid] = call
     return calls, skipped, keep
@@ -182,21 +186,31 @@ def run(reps=10, rounds=5, log=None, only=None, sustained=False):
 
 
 def write_rules(results, path=TABLE):
-    """Rewrite the RULES block: one exact-shape rule per class (dense)."""
-    lines = ["static const Rule kRules[] = {"]
+    """Rewrite the RULES block: one exact-shape rule per swept class.  Rules
+    of classes not in `results` are kept as they are."""
+    text = open(path).read()
+    m = re.search(r"// BEGIN RULES \(written by the sweep\)\n(.*?)// END RULES", text, flags=re.S)
+    old = {}
+    for line in m.group(1).splitlines():
+        c = re.search(r"//\s*([^:]+):", line)
+        if c and line.strip().startswith("{"):
+            old[c.group(1)] = line
+    new = {}
     for r in results:
-        lines.append(
+        new[r["class"]] = (
             f"    {{{r['M']}, {r['M']}, {r['N']}, {r['N']}, {r['K']}, {r['K']}, "
             f"{int(r['b_col'])}, {int(r.get('grouped', False))}, {r['best_id']}}},  "
             f"// {r['class']}: {r['best']} "
             f"{r['best_tflops']:.0f} TFLOP/s")
+    merged = dict(old)
+    merged.update(new)
+    lines = ["static const Rule kRules[] = {"] + list(merged.values())
     lines.append("    {0, 0, 0, 0, 0, 0, -1, -1, -1},  // sentinel")
     lines.append("};")
-    text = open(path).read()
-    new = re.sub(r"(// BEGIN RULES \(written by the sweep\)\n).*?(// END RULES)",
-                 lambda m: m.group(1) + "\n".join(lines) + "\n" + m.group(2), text, flags=re.S)
+    out = re.sub(r"(// BEGIN RULES \(written by the sweep\)\n).*?(// END RULES)",
+                 lambda mm: mm.group(1) + "\n".join(lines) + "\n" + mm.group(2), text, flags=re.S)
     with open(path, "w") as f:
-        f.write(new)
+        f.write(out)
 
 
 def main(argv=None):
@@ -208,8 +222,14 @@ def main(argv=None):
     ap.add_argument("--sustained", action="store_true",
                     help="back-to-back launches, no L2 flush")
     ap.add_argument("--write", action="store_true")
+    ap.add_argument("--from-log", default=None,
+                    help="write the rules from a saved --log file instead of sweeping")
     a = ap.parse_args(argv)
     sys.path.insert(0, ROOT)
+    if a.from_log:
+        with open(a.from_log) as f:
+            write_rules([json.loads(line) for line in f if line.strip()])
+        return
     res = run(a.reps, a.rounds, a.log, a.only, a.sustained)
     if a.write:
         write_rules(res)

@@ -197,10 +197,18 @@ def test_runs_on_a_side_stream():
 
 # --------------------------------------------------------------- grouped
 
+# 128 x 256 / 128 x 128 row tiles; swapped operands (one CTA, then CTA pairs)
+GROUPED_CONFIGS = [0, 1, 25, 26, 27]
+
+
 @pytest.mark.parametrize("b_col", [False, True])
 @pytest.mark.parametrize("out_f32", [False, True])
-@pytest.mark.parametrize("config", [0, 1])
+@pytest.mark.parametrize("config", GROUPED_CONFIGS)
 def test_grouped_every_element(b_col, out_f32, config):
+    if config >= 25:
+        assert dg.gemm_config_name(config).startswith("gswap")
+    if config >= 26:
+        assert dg.gemm_config_name(config).startswith("gswap2")
     rows_per = np.array([0, 3, 130, 1, 0, 257, 64, 0], dtype=np.int32)
     G, N, K = len(rows_per), 200, 136
     total = int(rows_per.sum())
@@ -229,14 +237,19 @@ def test_grouped_every_element(b_col, out_f32, config):
     g.check_canaries()
 
 
-def test_grouped_counts_beyond_total_are_clipped_and_reported():
+@pytest.mark.parametrize("config", [-1, 25, 26])
+def test_grouped_counts_beyond_total_are_clipped_and_reported(config):
     rows_per = np.array([5, 300, 40], dtype=np.int32)  # sums to 345
     total, N, K = 200, 64, 64                           # caller says 200
     X = torch.randn(total, K).bfloat16()
     W = torch.randn(3, K, N).bfloat16()
     g = Guarded(total, N, N, torch.bfloat16)
-    rc = dg.grouped_gemm(3, torch.from_numpy(rows_per).cuda(), total, N, K, X.cuda(), K,
-                         W.cuda(), N, K * N, g.ptr, N, None, 0, dg.GEMM_BF16)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        rc = dg.grouped_gemm(3, torch.from_numpy(rows_per).cuda(), total, N, K, X.cuda(), K,
+                             W.cuda(), N, K * N, g.ptr, N, None, 0, dg.GEMM_BF16)
+    finally:
+        dg.gemm_force_config(-1)
     assert rc == 0
     torch.cuda.synchronize()
     assert dg.gemm_device_status() == dg.GEMM_ERR_INVALID_ARG
@@ -245,6 +258,82 @@ def test_grouped_counts_beyond_total_are_clipped_and_reported():
     ref = oracle.grouped_gemm(np.array([5, 195], dtype=np.int32), N, K, X, K, W, N, K * N,
                               dtype="bf16", threads=THREADS)
     compare(g.matrix().double().cpu().numpy(), ref, 2, "clipped groups")
+
+
+def _grouped_problem(rows_per, N, K, seed, dtype=torch.bfloat16, b_col=False):
+    G = len(rows_per)
+    total = int(np.sum(rows_per))
+    gen = torch.Generator().manual_seed(seed)
+    X = torch.randn(total, K, generator=gen).to(dtype)
+    W = (torch.randn(*((G, N, K) if b_col else (G, K, N)), generator=gen) * 0.05).to(dtype)
+    bias = torch.randn(G, N, generator=gen).to(dtype)
+    return X, W, bias
+
+
+@pytest.mark.parametrize("config", [25, 26])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_grouped_swap_many_groups_every_element(config, dtype):
+    # 40 groups: empty, 1..15 rows (one 16-row box), exact multiples of 16,
+    # 256 (one full tile), 257 and 600 (two and three near-equal row blocks)
+    rng = np.random.default_rng(77)
+    rows_per = np.concatenate([[0, 1, 15, 16, 17, 255, 256, 257, 600, 0, 48, 112],
+                               rng.integers(0, 200, size=28)]).astype(np.int32)
+    N, K = 392, 200
+    name = "f16" if dtype == torch.float16 else "bf16"
+    X, W, bias = _grouped_problem(rows_per, N, K, seed=config, dtype=dtype)
+    total = int(rows_per.sum())
+    ref = oracle.grouped_gemm(rows_per, N, K, X, K, W, N, N * K, bias=bias, relu=True,
+                              dtype=name, threads=THREADS)
+    g = Guarded(total, N, N, dtype)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        rc = dg.grouped_gemm(len(rows_per), torch.from_numpy(rows_per).cuda(), total, N, K,
+                             X.cuda(), K, W.cuda(), N, N * K, g.ptr, N, bias.cuda(),
+                             dg.GEMM_EPI_BIAS | dg.GEMM_EPI_RELU,
+                             dg.GEMM_F16 if dtype == torch.float16 else dg.GEMM_BF16)
+    finally:
+        dg.gemm_force_config(-1)
+    assert rc == 0, dg.gemm_status_string(rc)
+    torch.cuda.synchronize()
+    assert dg.gemm_device_status() == 0
+    compare(g.matrix().double().cpu().numpy(), ref, 2, "grouped swap, 40 groups")
+    g.check_canaries()
+
+
+@pytest.mark.parametrize("config", [25, 26])
+def test_grouped_swap_tile_queue_resets_between_launches_and_streams(config):
+    # The tile queue's counter lives in each stream's scratch and every
+    # launch must leave it at 0: ten launches in a row on one stream, then
+    # two streams at once, each result checked in full.
+    rows_per = np.array([70, 0, 300, 5, 129], dtype=np.int32)
+    N, K = 256, 128
+    X, W, _ = _grouped_problem(rows_per, N, K, seed=9)
+    total = int(rows_per.sum())
+    ref = oracle.grouped_gemm(rows_per, N, K, X, K, W, N, N * K, dtype="bf16", threads=THREADS)
+    dX, dW, drows = X.cuda(), W.cuda(), torch.from_numpy(rows_per).cuda()
+    assert dg.gemm_force_config(config) == 0
+    try:
+        outs = []
+        for _ in range(10):
+            y = torch.empty(total, N, dtype=torch.bfloat16, device="cuda")
+            assert dg.grouped_gemm(5, drows, total, N, K, dX, K, dW, N, N * K, y, N, None, 0,
+                                   dg.GEMM_BF16) == 0
+            outs.append(y)
+        streams = [torch.cuda.Stream() for _ in range(2)]
+        torch.cuda.synchronize()
+        for st in streams:
+            with torch.cuda.stream(st):
+                for _ in range(3):
+                    y = torch.empty(total, N, dtype=torch.bfloat16, device="cuda")
+                    assert dg.grouped_gemm(5, drows, total, N, K, dX, K, dW, N, N * K, y, N,
+                                           None, 0, dg.GEMM_BF16) == 0
+                    outs.append(y)
+        torch.cuda.synchronize()
+    finally:
+        dg.gemm_force_config(-1)
+    assert dg.gemm_device_status() == 0
+    for i, y in enumerate(outs):
+        compare(y.double().cpu().numpy(), ref, 2, f"launch {i}")
 
 
 # -------------------------------------------------------------- watchdog
