@@ -328,8 +328,33 @@ def bench_ours(args, rank, local, world):
     e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
 
     peaks, peak_src = _peaks()
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    # Back-to-back launches for half a second or more run under the power cap:
+    # the tensor peak to compare with is then the sustained cuBLAS figure.
+    sustained = flush is None and total_ms >= 500.0
+    peak = float(peaks.get("bf16_tflops_sustained", burst)) if sustained else burst
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     achieved = flops / (ms_per_step * 1e-3) / 1e12
+    alg_bytes = in_bytes + out_bytes
+    # the roofline is the slower of the two bounds: FLOPs at the dense tensor
+    # peak, or the algorithmic bytes at the HBM copy bandwidth
+    t_tensor = flops / (peak * 1e12)
+    t_hbm = alg_bytes / (hbm * 1e9)
+    if t_hbm > t_tensor:
+        gbs = alg_bytes / (ms_per_step * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(gbs / hbm, 4), "peak_source": f"{peak_src} HBM copy bandwidth"}
+    else:
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} bf16 dense "
+                + ("(sustained: back-to-back launches under the power cap)" if sustained
+                   else "(burst)")
+                + ("; fp16 has the same dense rate" if w.dtype == "f16" else ""),
+                "frac_of_burst": round(achieved / burst, 4)}
+    roof["traffic"] = _traffic(w.name)
+    roof["algorithmic_bytes"] = alg_bytes
+    roof["bound_times_us"] = {"tensor": round(t_tensor * 1e6, 2), "hbm": round(t_hbm * 1e6, 2)}
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
@@ -346,11 +371,8 @@ def bench_ours(args, rank, local, world):
             "config_id": lib.gemm_select_config(w.M, w.N, w.K, code, epi) if not w.grouped
             else None,
         },
-        "pct_of_peak": round(100.0 * achieved / peak, 2),
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "peak_source": f"{peak_src} bf16 dense (burst)",
-                     "traffic": _traffic(w.name), "algorithmic_bytes": in_bytes + out_bytes},
+        "pct_of_peak": round(100.0 * achieved / burst, 2),
+        "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "steps": e2e_steps},
         "gpu_launches": args.steps,
