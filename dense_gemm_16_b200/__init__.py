@@ -34,6 +34,11 @@ GEMM_EPI_BIAS = 0x1
 GEMM_EPI_RELU = 0x2
 GEMM_B_COL_MAJOR = 0x100
 
+# trace events (gemm_set_trace): column of a block's row in the trace buffer
+(GEMM_TRACE_ENTRY, GEMM_TRACE_SETUP, GEMM_TRACE_FIRST_LOAD, GEMM_TRACE_FIRST_DATA,
+ GEMM_TRACE_LAST_MMA, GEMM_TRACE_FIRST_EPI, GEMM_TRACE_EPI_DONE, GEMM_TRACE_EXIT) = range(8)
+GEMM_TRACE_EVENTS = 8
+
 _lib = None
 _lock = threading.Lock()
 
@@ -80,6 +85,8 @@ def lib() -> ctypes.CDLL:
             L.conv2d_im2col.restype = I
             L.gemm_splitk_noalloc.argtypes = [I, I, I, P, L64, P, L64, P, L64, P, U, I, I, P]
             L.gemm_splitk_noalloc.restype = I
+            L.gemm_set_trace.argtypes = [P, L64]
+            L.gemm_set_trace.restype = I
             _lib = L
     return _lib
 
@@ -154,6 +161,12 @@ def gemm_version() -> str:
 
 def gemm_device_status(stream=None, clear: bool = True) -> int:
     return lib().gemm_device_status(_stream(stream), int(clear))
+
+
+def gemm_set_trace(buffer, nbytes: int) -> int:
+    """C-ABI ``gemm_set_trace``: per-block event times of later launches go
+    to ``buffer`` (device memory, ``nbytes`` long); ``None`` turns tracing off."""
+    return lib().gemm_set_trace(_ptr(buffer), nbytes)
 
 
 def gemm_set_timeout_ns(ns: int) -> int:

@@ -44,6 +44,9 @@ static const Config kConfigs[] = {
     {"gswap_128x256_s4", kKindGroupedSwap, 256, 4, 1, 1, 0, 0},
     {"gswap2_256x256_s6", kKindGroupedSwapPair, 256, 6, 1, 1, 0, 0},
     {"gswap2_256x256_s6_xl", kKindGroupedSwapPair, 256, 6, 1, 1, 0, 2},
+    {"tc1_128x64_s8_g8", kKindSingle, 64, 8, 8, 1, 2, 2},
+    {"tc1_128x64_s8_g8_sk", kKindSingle, 64, 8, 8, -1, 2, 2},
+    {"tc1_128x64_s8_g8_k2", kKindSingle, 64, 8, 8, 2, 2, 2},
 };
 static constexpr int kNumConfigs = static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0]));
 
@@ -58,14 +61,14 @@ struct Rule {
 
 // BEGIN RULES (written by the sweep)
 static const Rule kRules[] = {
-    {256, 256, 256, 256, 256, 256, 0, 0, 1},  // square256: tc1_128x128_s6_g8 3 TFLOP/s
-    {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 1},  // m1024n1024k2048: tc1_128x128_s6_g8 215 TFLOP/s
+    {256, 256, 256, 256, 256, 256, 0, 0, 28},  // square256: tc1_128x64_s8_g8 3 TFLOP/s
+    {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 8},  // m1024n1024k2048: tc1_128x128_s6_g8_k2 210 TFLOP/s
     {2048, 2048, 2048, 2048, 2048, 2048, 0, 0, 0},  // square2048: tc1_128x256_s4_g8 714 TFLOP/s
     {4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 11},  // square4096 (sustained): pair_256x256_s6_g16 1285 TFLOP/s
     {8192, 8192, 8192, 8192, 8192, 8192, 0, 0, 13},  // square8192 (sustained): pair_256x512_s4_g16 1311 TFLOP/s
-    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 16},  // m1000n1000k2000_bcol: tc1_128x128_s6_g8_pn 186 TFLOP/s
-    {4096, 4096, 4096, 4096, 512, 512, 1, 0, 1},  // m4096n4096k512_bcol: tc1_128x128_s6_g8 509 TFLOP/s
-    {16, 16, 8192, 8192, 8192, 8192, 1, 0, 6},  // m16n8192k8192_bcol: swap_128x16_s8_k4 61 TFLOP/s
+    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 28},  // m1000n1000k2000_bcol: tc1_128x64_s8_g8 195 TFLOP/s
+    {4096, 4096, 4096, 4096, 512, 512, 1, 0, 0},  // m4096n4096k512_bcol: tc1_128x256_s4_g8 599 TFLOP/s
+    {16, 16, 8192, 8192, 8192, 8192, 1, 0, 21},  // m16n8192k8192_bcol: swap_128x16_s8_sk 62 TFLOP/s
     {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 704 TFLOP/s
     {16384, 16384, 4096, 4096, 4096, 4096, 0, 1, 0},  // moe8_n4096_k4096: tc1_128x256_s4_g8 1228 TFLOP/s
     {8192, 8192, 768, 768, 2048, 2048, 0, 1, 27},  // moe64_n768_k2048: gswap2_256x256_s6_xl 331 TFLOP/s

@@ -37,6 +37,7 @@ struct Config {
 // Each returns {nullptr, 0} for a combination that was not compiled.
 KernelEntry kernels_bn256(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_bn128(bool q_mn, bool bf16, bool out_f32, bool grouped);
+KernelEntry kernels_bn64(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_swap(int bn, bool bf16, bool out_f32);
 KernelEntry kernels_pair(int bn, int stages, bool q_mn, bool bf16, bool out_f32);
 KernelEntry kernels_tf32(int bn, bool q_mn);

@@ -53,6 +53,15 @@ constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
 constexpr int kMaxDevices = 64;
 
 std::atomic<unsigned long long> g_timeout_ns{kDefaultTimeoutNs};
+// gemm_set_trace: the caller's trace buffer and how many blocks it holds
+std::atomic<unsigned long long*> g_trace{nullptr};
+std::atomic<int> g_trace_blocks{0};
+
+// Stamp the current trace setting into a launch's parameters.
+void set_trace(KParams& kp) {
+  kp.trace = g_trace.load();
+  kp.trace_blocks = kp.trace ? g_trace_blocks.load() : 0;
+}
 std::atomic<int> g_forced_config{-1};
 
 struct DeviceState {
@@ -318,6 +327,7 @@ KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool gro
   }
   if (c.bn == 256) return kernels_bn256(q_mn, bf16, f32, grouped);
   if (c.bn == 128) return kernels_bn128(q_mn, bf16, f32, grouped);
+  if (c.bn == 64) return kernels_bn64(q_mn, bf16, f32, grouped);
   return {nullptr, 0};
 }
 
@@ -339,8 +349,10 @@ int launch(const KernelEntry& k, int grid, cudaStream_t stream, const CUtensorMa
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
+  KParams kpt = kp;
+  set_trace(kpt);
   void* args[4] = {const_cast<CUtensorMap*>(&tp), const_cast<CUtensorMap*>(&tq),
-                   const_cast<CUtensorMap*>(&tc), const_cast<KParams*>(&kp)};
+                   const_cast<CUtensorMap*>(&tc), &kpt};
   cudaError_t e = cudaLaunchKernelExC(&cfg, k.fn, args);
   return e == cudaSuccess ? GEMM_OK : cuda_fail(e);
 }
@@ -749,6 +761,7 @@ int launch_grouped_swap(DeviceState* ds, const KernelEntry& k, const Config& cfg
   kp.pol_p = cfg.pol_p;
   kp.pol_q = cfg.pol_q;
   kp.counters = counters + kCounterSlots;  // the tile-queue counter
+  set_trace(kp);
   const bool pair = cfg.kind == kKindGroupedSwapPair;
   const long long cols = pair ? 2 * kBM : kBM;
   const long long nb = (N + cols - 1) / cols;
@@ -896,6 +909,19 @@ int gemm_device_status(void* stream_, int clear) {
   if (w == kStatusOk) return GEMM_OK;
   if (w == kStatusBadGroups) return GEMM_ERR_INVALID_ARG;
   return GEMM_ERR_DEVICE_TIMEOUT;
+}
+
+int gemm_set_trace(void* buffer, int64_t bytes) {
+  if (buffer && (reinterpret_cast<uintptr_t>(buffer) & 7u) != 0) return GEMM_ERR_MISALIGNED;
+  const int64_t blocks = buffer ? bytes / static_cast<int64_t>(8 * kTraceEvents) : 0;
+  if (blocks <= 0) {
+    g_trace.store(nullptr);
+    g_trace_blocks.store(0);
+    return GEMM_OK;
+  }
+  g_trace_blocks.store(static_cast<int>(std::min<int64_t>(blocks, INT32_MAX)));
+  g_trace.store(static_cast<unsigned long long*>(buffer));
+  return GEMM_OK;
 }
 
 uint64_t gemm_set_timeout_ns(uint64_t ns) {

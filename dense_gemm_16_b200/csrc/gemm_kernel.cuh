@@ -47,7 +47,7 @@ template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT, bool SWAP,
           bool TF32 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                   const __grid_constant__ CUtensorMap tmC, const KParams p) {
+                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ KParams p) {
   using InT = typename std::conditional<
       TF32, float, typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type>::type;
   constexpr int ELEM = TF32 ? 4 : 2;           // input bytes
@@ -61,10 +61,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t P_BYTES = kBM * 128;     // 128 rows x one 128-byte K row
   constexpr uint32_t Q_BYTES = BN * 128;
   constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
-  // Swapped (skinny) tiles have a tiny MMA-N, so one accumulator would chain
-  // every MMA of a tile through its latency: consecutive K blocks rotate over
-  // NACC independent accumulators instead, summed in order by the epilogue.
-  constexpr int NACC = SWAP ? (BN <= 16 ? 4 : 2) : 1;
+  // Swapped (skinny) tiles have a tiny MMA-N, so chaining a tile's MMAs into
+  // one accumulator would pay each MMA's full latency: consecutive MMAs (the
+  // 32-byte K slices, across K blocks) rotate over NACC independent
+  // accumulators instead, summed in order by the epilogue.
+  constexpr int NACC = SWAP ? (BN <= 16 ? 8 : 4) : 1;
   constexpr int ACC_COLS = NACC * BN;  // TMEM columns per accumulator buffer
   constexpr uint32_t TMEM_COLS = (2 * ACC_COLS <= 32) ? 32 : (2 * ACC_COLS <= 64) ? 64
                                  : (2 * ACC_COLS <= 128) ? 128 : (2 * ACC_COLS <= 256) ? 256 : 512;
@@ -94,6 +95,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) trace_mark(p, kTrEntry);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -147,6 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
+  if (threadIdx.x == 0) trace_mark(p, kTrSetup);
 
   long long num_tiles = p.num_tiles;
   if constexpr (GROUPED) num_tiles = gt->tile_start[p.num_groups];
@@ -189,6 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_3d(qdst, &tmQ, kb * KB_EL, q0, c.zq, fb, pol_q);
           }
+          if (it == 0) trace_mark(p, kTrFirstLoad);
         }
       }
       if (!ok) {
@@ -216,15 +220,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + a * ACC_COLS;
         for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
-          const int r = (kb - w.kb0) % NACC;            // accumulator of this K block
-          const uint32_t d = d0 + static_cast<uint32_t>(r * BN);
-          const bool fresh = kb - w.kb0 < NACC;         // its first K block
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_phase(smem_u32(&full_bar[s]), ph, ctl, p, kStatusTimeoutMma)) {
             ok = false;
             break;
           }
+          if (it == 0) trace_mark(p, kTrFirstData);
           tc_fence_after();
           const uint32_t pbase = smem_u32(sP + s * P_BYTES);
           const uint32_t qbase = smem_u32(sQ + s * Q_BYTES);
@@ -240,16 +242,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 Q_MN ? (TF32 ? sw128_desc(qbase + k * MMA_K * 128, KB_EL * 128, 512, 1)
                              : sw128_desc(qbase + k * MMA_K * 128, KB_EL * 128, 1024))
                      : sw128_desc(qbase + k * 32, 16, 1024);
+            // MMA number `step` of the tile goes to accumulator step % NACC;
+            // the first NACC of them start their accumulator from zero
+            const int step = (kb - w.kb0) * 4 + k;
+            const uint32_t d = d0 + static_cast<uint32_t>((step % NACC) * BN);
+            const uint32_t acc = step >= NACC ? 1u : 0u;
             if constexpr (TF32)
-              mma_tf32<1>(d, adesc, bdesc, IDESC, (!fresh || k != 0) ? 1u : 0u);
+              mma_tf32<1>(d, adesc, bdesc, IDESC, acc);
             else
-              mma_f16<1>(d, adesc, bdesc, IDESC, (!fresh || k != 0) ? 1u : 0u);
+              mma_f16<1>(d, adesc, bdesc, IDESC, acc);
           }
           mma_commit<1>(smem_u32(&empty_bar[s]));  // frees the stage when read
         }
         if (!ok) break;
         mma_commit<1>(smem_u32(&accf_bar[a]));  // accumulator ready
       }
+      trace_mark(p, kTrLastMma);
       // every MMA this thread issued has completed before tensor memory is freed
       mma_commit<1>(smem_u32(drain_bar));
       wait_phase_drain(smem_u32(drain_bar), 0, 50000000ull);
@@ -287,6 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else if (!__all_sync(0xffffffffu, ok)) {
         break;
       }
+      if (warp == 2 && lane == 0 && local == 0) trace_mark(p, kTrFirstEpi);
       tc_fence_after();
       const int prow = c.p0 + row_local;  // this thread's accumulator row
       const int q0 = c.q0 * BN;
@@ -299,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                : bias + static_cast<long long>(c.group) * p.stride_bias);
       const uint32_t taddr =
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * ACC_COLS;
-      const TmemSrc tsrc{taddr, min(NACC, w.kb1 - w.kb0), BN};
+      const TmemSrc tsrc{taddr, min(NACC, 4 * (w.kb1 - w.kb0)), BN};
       bool finish = true;  // this block stores the tile
       const float* tile0 = nullptr;
       if (w.count > 1) {
@@ -377,9 +386,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_u32(&acce_bar[a]));
       }
     }
-    // every TMA store has finished with shared memory (and the output is
-    // written) before the block retires
-    if (TMA_EPI && lane == 0) tma_store_wait_all<0>();
+    // every TMA store has finished reading shared memory before the block
+    // retires; the writes themselves complete before the grid does
+    if (TMA_EPI && lane == 0) tma_store_wait_read<0>();
+    if (warp == 2 && lane == 0) trace_mark(p, kTrEpiDone);
   }
 
   tc_fence_before();
@@ -389,6 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc<1>(tmem_base, TMEM_COLS);
   }
+  if (threadIdx.x == 0) trace_mark(p, kTrExit);
 }
 
 // Shared memory a kernel instance needs (bytes, including alignment slack).

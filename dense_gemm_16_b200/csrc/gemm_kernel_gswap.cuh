@@ -107,7 +107,7 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, SharedC
 template <int TOK, int STAGES, bool P_MN, bool IN_BF16, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_gswap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ RowMaps tmX,
-                      const KParams p) {
+                      const __grid_constant__ KParams p) {
   using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
   constexpr uint32_t W_BYTES = kBM * 128;        // 128 columns of W x 64 K
   static_assert(TOK % 64 == 0 && TOK >= 128 && TOK <= 256, "row blocks of 128..256 rows");
@@ -136,6 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) trace_mark(p, kTrEntry);
   const int num_nb = (p.N + kBM - 1) / kBM;
 
   if (threadIdx.x == 0) {
@@ -190,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   const int num_tiles = gt->tile_start[p.num_groups];
+  if (threadIdx.x == 0) trace_mark(p, kTrSetup);
 
   if (warp == 0) {
     // ------------------------------------------- tile queue + TMA producer
@@ -298,6 +300,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         mma_commit<1>(smem_u32(&accf_bar[a]));
       }
+      trace_mark(p, kTrLastMma);
       mma_commit<1>(smem_u32(drain_bar));
       wait_phase_drain(smem_u32(drain_bar), 0, 50000000ull);
     }
@@ -360,6 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc<1>(tmem_base, TMEM_COLS);
   }
+  if (threadIdx.x == 0) trace_mark(p, kTrExit);
 }
 
 // ---------------------------------------------------------------------------
@@ -386,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int TOK, int STAGES, bool P_MN, bool IN_BF16, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_gswap2_kernel(const __grid_constant__ CUtensorMap tmW,
-                       const __grid_constant__ RowMaps tmX, const KParams p) {
+                       const __grid_constant__ RowMaps tmX, const __grid_constant__ KParams p) {
   using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
   static_assert(TOK % 64 == 0 && TOK >= 128 && TOK <= 256, "row blocks of 128..256 rows");
   constexpr int COLS = 2 * kBM;                     // output columns per pair tile
@@ -416,6 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) trace_mark(p, kTrEntry);
   const uint32_t rank = cluster_ctarank();  // 0 = leader
   const uint32_t peer = rank ^ 1u;
   const int num_nb = (p.N + COLS - 1) / COLS;
@@ -473,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   const int num_tiles = gt->tile_start[p.num_groups];
+  if (threadIdx.x == 0) trace_mark(p, kTrSetup);
   const uint32_t tqe_leader0 = map_shared_rank(smem_u32(&tqe_bar[0]), 0);
 
   if (warp == 0) {
@@ -609,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit<2>(smem_u32(&accf_bar[a]));
         mma_commit<2>(peer_accf0 + a * 8u);
       }
+      trace_mark(p, kTrLastMma);
       mma_commit<2>(smem_u32(drain_bar));
       wait_phase_drain(smem_u32(drain_bar), 0, 50000000ull);
     }
@@ -675,6 +682,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc<2>(tmem_base, TMEM_COLS);
   }
+  if (threadIdx.x == 0) trace_mark(p, kTrExit);
 }
 
 template <int TOK, int STAGES>

@@ -34,7 +34,7 @@ namespace dg16 {
 template <int BN, int NSUB, int STAGES, bool Q_MN, bool IN_BF16, typename OutT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
-                    const __grid_constant__ CUtensorMap tmC, const KParams p) {
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ KParams p) {
   using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
   constexpr int HALF_N = BN / 2;
   constexpr int TILE_N = BN * NSUB;                 // output columns per pair tile
@@ -71,6 +71,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // names the same barrier role in either CTA.
   const long long pair_id = blockIdx.x >> 1;
   const long long num_pairs = gridDim.x >> 1;
+  if (threadIdx.x == 0) trace_mark(p, kTrEntry);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -101,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   const long long num_tiles = p.num_tiles;
+  if (threadIdx.x == 0) trace_mark(p, kTrSetup);
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (both CTAs)
@@ -143,6 +145,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_3d_pair(qdst, &tmQ, kb * kBK, qc, zq, fb_leader, pol_q);
             }
           }
+          if (it == 0) trace_mark(p, kTrFirstLoad);
         }
       }
       if (!ok) {
@@ -179,6 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (it == 0) trace_mark(p, kTrFirstData);
           tc_fence_after();
           const uint32_t pbase = smem_u32(sP + s * P_BYTES);
           const uint32_t qbase = smem_u32(sQ + s * Q_BYTES);
@@ -201,6 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit<2>(smem_u32(&accf_bar[a]));
         mma_commit<2>(peer_accf0 + a * 8u);
       }
+      trace_mark(p, kTrLastMma);
       mma_commit<2>(smem_u32(drain_bar));
       wait_phase_drain(smem_u32(drain_bar), 0, 50000000ull);
     }
@@ -223,6 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t aph = ACC_BUFS == 2 ? ((local >> 1) & 1u) : (local & 1u);
       const bool ok = wait_phase<true>(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
+      if (warp == 2 && lane == 0 && local == 0) trace_mark(p, kTrFirstEpi);
       tc_fence_after();
       const int row0 = pb * (2 * kBM) + static_cast<int>(rank) * kBM + quad * 32;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * TILE_N;
@@ -237,7 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader0 + a * 8u);
     }
-    if (lane == 0) tma_store_wait_all<0>();
+    if (lane == 0) tma_store_wait_read<0>();  // staging read; writes finish with the grid
+    if (warp == 2 && lane == 0) trace_mark(p, kTrEpiDone);
   }
 
   tc_fence_before();
@@ -248,6 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc<2>(tmem_base, TMEM_COLS);
   }
+  if (threadIdx.x == 0) trace_mark(p, kTrExit);
 }
 
 template <int BN, int NSUB, int STAGES>

@@ -70,9 +70,26 @@ struct KParams {
   int z_p, z_q;           // 1: the P / Q operand advances with the batch
   long long stride_c;     // elements between batches' outputs
   long long stride_bias;  // elements between batches' bias vectors
+  // Optional tracing: when non-null, blocks below trace_blocks write the
+  // global timer at each event into trace[block * kTraceEvents + event].
+  unsigned long long* trace;
+  int trace_blocks;
+};
+
+// Trace events (the same numbering as the GEMM_TRACE_* constants of the C ABI).
+enum : int {
+  kTrEntry = 0, kTrSetup = 1, kTrFirstLoad = 2, kTrFirstData = 3,
+  kTrLastMma = 4, kTrFirstEpi = 5, kTrEpiDone = 6, kTrExit = 7, kTraceEvents = 8
 };
 
 enum : int { kPolicyNormal = 0, kPolicyFirst = 1, kPolicyLast = 2 };
+
+// Record the global timer for trace event `ev` of this block (one thread
+// calls it; a no-op unless tracing is on).
+__device__ __forceinline__ void trace_mark(const KParams& p, int ev) {
+  if (p.trace != nullptr && static_cast<int>(blockIdx.x) < p.trace_blocks)
+    p.trace[static_cast<long long>(blockIdx.x) * kTraceEvents + ev] = global_timer_ns();
+}
 
 __device__ __forceinline__ uint64_t make_policy(int code) {
   return code == kPolicyLast ? policy_evict_last()
@@ -289,29 +306,6 @@ __device__ __forceinline__ void put_partial16(float* tile, int row, int cc, cons
                        __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
 }
 
-// Columns cc .. cc+15 of this thread's row summed over `count` partial tiles
-// `stride` floats apart, in piece order (so the result does not depend on
-// which block finished last); returned as raw fp32 bits.
-__device__ __forceinline__ void sum_partials16(const float* tile0, long long stride, int count,
-                                               int row, int cc, uint32_t (&out)[16]) {
-  float f[16];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) f[j] = 0.0f;
-  for (int s = 0; s < count; ++s) {
-    const float4* q = reinterpret_cast<const float4*>(tile0 + s * stride);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 v = __ldcg(q + (static_cast<long long>(cc / 4 + j) * kBM + row));
-      f[4 * j] += v.x;
-      f[4 * j + 1] += v.y;
-      f[4 * j + 2] += v.z;
-      f[4 * j + 3] += v.w;
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 16; ++j) out[j] = __float_as_uint(f[j]);
-}
-
 // Epilogue for one accumulator row held by this thread, from any source of
 // raw fp32 values: src.get<16>(cc, v) fills v[0..15] with columns cc .. cc+15
 // of the row (a warp-collective TMEM load, or a partial-tile sum).  Output row
@@ -328,13 +322,18 @@ __device__ __forceinline__ void store_rows_from(Src&& src, int prow, int row_end
   for (int cc = 0; cc < TILE_N; cc += 16) {
     const int col0 = q0 + cc;
     if (col0 >= p.N) break;  // warp-uniform
+    // the bias loads go out before the accumulator read, so their latency overlaps it
+    float bv[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      bv[j] = (bias_g != nullptr && col0 + j < p.N) ? to_f32<InT>(bias_g[col0 + j]) : 0.0f;
     uint32_t v[16];
     src.template get<16>(cc, v);
     float f[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       float x = __uint_as_float(v[j]);
-      if (bias_g != nullptr && col0 + j < p.N) x += to_f32<InT>(bias_g[col0 + j]);
+      if (bias_g != nullptr) x += bv[j];
       if (relu) x = fmaxf(x, 0.0f);
       f[j] = x;
     }
@@ -390,6 +389,11 @@ __device__ __forceinline__ void store_tma_from(Src&& src, int row0, int q0, int 
   for (int c0 = 0; c0 < TILE_N; c0 += CH) {
     const int col0 = q0 + c0;
     if (col0 >= p.N) break;  // warp-uniform
+    // the bias loads go out before the accumulator read, so their latency overlaps it
+    float bv[CH];
+#pragma unroll
+    for (int j = 0; j < CH; ++j)
+      bv[j] = (bias != nullptr && col0 + j < p.N) ? to_f32<InT>(bias[col0 + j]) : 0.0f;
     uint32_t v[CH];
     src.template get<CH>(c0, v);
     uint32_t packed[32];
@@ -398,8 +402,8 @@ __device__ __forceinline__ void store_tma_from(Src&& src, int row0, int q0, int 
       for (int j = 0; j < 32; ++j) {
         float x0 = __uint_as_float(v[2 * j]), x1 = __uint_as_float(v[2 * j + 1]);
         if (bias != nullptr) {
-          if (col0 + 2 * j < p.N) x0 += to_f32<InT>(bias[col0 + 2 * j]);
-          if (col0 + 2 * j + 1 < p.N) x1 += to_f32<InT>(bias[col0 + 2 * j + 1]);
+          x0 += bv[2 * j];
+          x1 += bv[2 * j + 1];
         }
         if (relu) {
           x0 = fmaxf(x0, 0.0f);
@@ -411,7 +415,7 @@ __device__ __forceinline__ void store_tma_from(Src&& src, int row0, int q0, int 
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         float x = __uint_as_float(v[j]);
-        if (bias != nullptr && col0 + j < p.N) x += to_f32<InT>(bias[col0 + j]);
+        if (bias != nullptr) x += bv[j];
         if (relu) x = fmaxf(x, 0.0f);
         packed[j] = __float_as_uint(x);
       }
@@ -491,11 +495,33 @@ struct PartialSrc {
   const float* tile0;
   long long stride;
   int count, row;
+  // Columns cc .. cc+W-1 of this thread's row summed over the `count` partial
+  // tiles `stride` floats apart, in piece order (so the result does not
+  // depend on which block finished last); returned as raw fp32 bits.  All W/4
+  // loads of one piece are issued before any is used, so a piece costs one
+  // memory round trip, not W/4.
   template <int W>
   __device__ __forceinline__ void get(int cc, uint32_t (&v)[W]) const {
+    static_assert(W % 16 == 0, "whole 16-column groups");
+    float f[W];
 #pragma unroll
-    for (int h = 0; h < W; h += 16)
-      sum_partials16(tile0, stride, count, row, cc + h, *reinterpret_cast<uint32_t(*)[16]>(&v[h]));
+    for (int j = 0; j < W; ++j) f[j] = 0.0f;
+    for (int s = 0; s < count; ++s) {
+      const float4* q = reinterpret_cast<const float4*>(tile0 + s * stride);
+      float4 t[W / 4];
+#pragma unroll
+      for (int j = 0; j < W / 4; ++j)
+        t[j] = __ldcg(q + (static_cast<long long>(cc / 4 + j) * kBM + row));
+#pragma unroll
+      for (int j = 0; j < W / 4; ++j) {
+        f[4 * j] += t[j].x;
+        f[4 * j + 1] += t[j].y;
+        f[4 * j + 2] += t[j].z;
+        f[4 * j + 3] += t[j].w;
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < W; ++j) v[j] = __float_as_uint(f[j]);
   }
 };
 

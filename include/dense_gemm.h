@@ -228,6 +228,37 @@ GEMM_API uint64_t gemm_set_timeout_ns(uint64_t ns);
  */
 GEMM_API int gemm_watchdog_selftest(uint64_t timeout_ns, void* stream);
 
+/* ---- tracing ----------------------------------------------------------- */
+
+/* Events a traced launch records per block (indices into its row). */
+enum {
+  GEMM_TRACE_ENTRY = 0,      /* the block started */
+  GEMM_TRACE_SETUP = 1,      /* barriers, tensor memory and tables ready */
+  GEMM_TRACE_FIRST_LOAD = 2, /* the producer issued its first copy */
+  GEMM_TRACE_FIRST_DATA = 3, /* the MMA issuer saw its first full stage */
+  GEMM_TRACE_LAST_MMA = 4,   /* the MMA issuer committed its last accumulator */
+  GEMM_TRACE_FIRST_EPI = 5,  /* the first epilogue warp got its first accumulator */
+  GEMM_TRACE_EPI_DONE = 6,   /* that warp finished its last tile (stores issued) */
+  GEMM_TRACE_EXIT = 7,       /* the block is about to return */
+  GEMM_TRACE_EVENTS = 8
+};
+
+/*
+ * gemm_set_trace -- record where launches spend their time.  `buffer` is
+ * caller-owned device memory of `bytes` bytes; NULL (or bytes too small for
+ * one block) turns tracing off, which is the default.  While it is set,
+ * every GEMM kernel launched by this library writes, for each block b below
+ * bytes / (8 * GEMM_TRACE_EVENTS), the device's global timer (nanoseconds,
+ * uint64) at event e into buffer[b * GEMM_TRACE_EVENTS + e].  Events a block
+ * never reaches (a block with no tile has no FIRST_DATA) keep their old
+ * value, so zero the buffer before the launch of interest.  Every launch
+ * overwrites the rows of its blocks, so trace one launch at a time.  The
+ * setting is process-wide and not synchronised with launches in flight.
+ * Returns GEMM_OK, or GEMM_ERR_MISALIGNED for a buffer that is not 8-byte
+ * aligned.
+ */
+GEMM_API int gemm_set_trace(void* buffer, int64_t bytes);
+
 /* ---- tile configurations (the offline sweep's table) ------------------- */
 
 /* Number of tile configurations compiled into the library. */

@@ -201,3 +201,11 @@ def test_batched_empty_is_a_noop():
 ])
 def test_conv_argument_errors(args, expect):
     assert dg.lib().conv2d_im2col(*args, None) == expect
+
+
+def test_trace_setting_checks_alignment_and_turns_off():
+    # no GPU needed: the call only records the buffer
+    assert dg.gemm_set_trace(0x1003, 4096) == dg.GEMM_ERR_MISALIGNED
+    assert dg.gemm_set_trace(None, 0) == dg.GEMM_OK
+    assert dg.gemm_set_trace(0x1000, 8) == dg.GEMM_OK  # too small for one block: off
+    assert dg.GEMM_TRACE_EVENTS == 8 and dg.GEMM_TRACE_EXIT == 7

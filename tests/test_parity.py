@@ -73,7 +73,7 @@ def test_moe_grouped_sampled():
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("b_col", [False, True])
-@pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 12, 13, 23, 24])
+@pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 12, 13, 23, 24, 28, 29, 30])
 def test_exact_integers(dtype, b_col, config):
     """Integer inputs in [-2, 2] with K <= 4096: every partial sum is an
     exact integer below 2^24, so the fp32 accumulator is exact in any order
@@ -144,7 +144,10 @@ def test_empty_m_or_n_is_a_noop():
     assert bool((g.ibuf.cpu() == g.sent).all())
 
 
-@pytest.mark.parametrize("config", range(25))
+DENSE_CONFIGS = list(range(25)) + [28, 29, 30]  # 25..27 are grouped-only
+
+
+@pytest.mark.parametrize("config", DENSE_CONFIGS)
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("out_f32", [False, True])
 def test_every_config_on_ragged_problem(config, dtype, out_f32):
@@ -181,6 +184,65 @@ def test_swap_config_rejects_row_major_b():
                        dg.GEMM_F16) == dg.GEMM_ERR_UNSUPPORTED
     finally:
         dg.gemm_force_config(-1)
+
+
+def test_configs_of_the_other_kind_are_rejected():
+    # a grouped-only config on a dense call, a CTA-pair dense config on a
+    # grouped call: UNSUPPORTED, and nothing is written
+    A = torch.ones(64, 64, dtype=torch.half, device="cuda")
+    B = torch.ones(64, 64, dtype=torch.half, device="cuda")
+    C = torch.zeros(64, 64, dtype=torch.half, device="cuda")
+    rows = torch.tensor([32, 32], dtype=torch.int32, device="cuda")
+    Bg = torch.ones(2, 64, 64, dtype=torch.half, device="cuda")
+    pair = [i for i in range(dg.gemm_num_configs()) if dg.gemm_config_name(i).startswith("pair")][0]
+    try:
+        assert dg.gemm_force_config(25) == 0
+        assert dg.gemm(64, 64, 64, A, 64, B, 64, C, 64, None, 0,
+                       dg.GEMM_F16) == dg.GEMM_ERR_UNSUPPORTED
+        assert dg.gemm_force_config(pair) == 0
+        assert dg.grouped_gemm(2, rows, 64, 64, 64, A, 64, Bg, 64, 64 * 64, C, 64, None, 0,
+                               dg.GEMM_F16) == dg.GEMM_ERR_UNSUPPORTED
+    finally:
+        dg.gemm_force_config(-1)
+    torch.cuda.synchronize()
+    assert int(C.abs().sum()) == 0
+
+
+@pytest.mark.parametrize("config", [1, 13, 21, 8])  # single CTA, pair, swapped stream-K, split-K
+def test_trace_records_ordered_events_per_block(config):
+    M, N, K = (16, 8192, 1024) if config == 21 else (1024, 1024, 512)
+    A = torch.randn(M, K, dtype=torch.half, device="cuda")
+    B = torch.randn(N, K, dtype=torch.half, device="cuda")
+    C = torch.empty(M, N, dtype=torch.half, device="cuda")
+    buf = torch.zeros(148 * dg.GEMM_TRACE_EVENTS, dtype=torch.int64, device="cuda")
+    assert dg.gemm_set_trace(buf, buf.numel() * 8) == 0
+    assert dg.gemm_force_config(config) == 0
+    try:
+        assert dg.gemm(M, N, K, A, K, B, K, C, N, None, dg.GEMM_B_COL_MAJOR, dg.GEMM_F16) == 0
+        torch.cuda.synchronize()
+    finally:
+        dg.gemm_force_config(-1)
+        dg.gemm_set_trace(None, 0)
+    t = buf.view(148, dg.GEMM_TRACE_EVENTS).cpu().numpy()
+    started = t[:, dg.GEMM_TRACE_ENTRY] > 0
+    assert started.sum() > 0
+    for row in t[started]:
+        assert row[dg.GEMM_TRACE_ENTRY] <= row[dg.GEMM_TRACE_SETUP] <= row[dg.GEMM_TRACE_EXIT]
+        if row[dg.GEMM_TRACE_FIRST_DATA] > 0:  # a block with work
+            assert row[dg.GEMM_TRACE_SETUP] <= row[dg.GEMM_TRACE_FIRST_LOAD]
+            assert row[dg.GEMM_TRACE_FIRST_LOAD] <= row[dg.GEMM_TRACE_FIRST_DATA]
+            assert row[dg.GEMM_TRACE_FIRST_DATA] <= row[dg.GEMM_TRACE_LAST_MMA] <= row[dg.GEMM_TRACE_EXIT]
+        if row[dg.GEMM_TRACE_FIRST_EPI] > 0:
+            assert row[dg.GEMM_TRACE_FIRST_EPI] <= row[dg.GEMM_TRACE_EPI_DONE] <= row[dg.GEMM_TRACE_EXIT]
+    # tracing changes no result: the same call untraced gives the same bits
+    C2 = torch.empty_like(C)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        assert dg.gemm(M, N, K, A, K, B, K, C2, N, None, dg.GEMM_B_COL_MAJOR, dg.GEMM_F16) == 0
+        torch.cuda.synchronize()
+    finally:
+        dg.gemm_force_config(-1)
+    assert torch.equal(C, C2)
 
 
 def test_runs_on_a_side_stream():
