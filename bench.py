@@ -205,9 +205,11 @@ def time_oracle(w, budget_s: float = 12.0, threads: int | None = None):
             oracle.gemm_at(w.M, w.N, w.K, A, w.K, B, ldb, r, c, b_colmajor=w.b_colmajor,
                            bias=bias, relu=w.relu, dtype=w.dtype, threads=threads)
             return time.perf_counter() - t0
-    n = max(used, 64)
+    # calibrate on a sample large enough that per-call overheads do not
+    # inflate the per-element estimate, then size the timed sample to the budget
+    n = max(used * 64, 4096)
     dt = run(n)
-    n = int(min(max(n, n * budget_s / max(dt, 1e-3)), 2_000_000))
+    n = int(min(max(n, n * budget_s / max(dt, 1e-3)), 4_000_000))
     dt = run(n)
     return 2.0 * w.K * n / dt / 1e12, dt, n, used
 
