@@ -62,12 +62,12 @@ struct Rule {
 // BEGIN RULES (written by the sweep)
 static const Rule kRules[] = {
     {256, 256, 256, 256, 256, 256, 0, 0, 28},  // square256: tc1_128x64_s8_g8 3 TFLOP/s
-    {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 8},  // m1024n1024k2048: tc1_128x128_s6_g8_k2 210 TFLOP/s
-    {2048, 2048, 2048, 2048, 2048, 2048, 0, 0, 0},  // square2048: tc1_128x256_s4_g8 714 TFLOP/s
+    {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 28},  // m1024n1024k2048: tc1_128x64_s8_g8 209 TFLOP/s
+    {2048, 2048, 2048, 2048, 2048, 2048, 0, 0, 0},  // square2048: tc1_128x256_s4_g8 672 TFLOP/s
     {4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 11},  // square4096 (sustained): pair_256x256_s6_g16 1285 TFLOP/s
     {8192, 8192, 8192, 8192, 8192, 8192, 0, 0, 13},  // square8192 (sustained): pair_256x512_s4_g16 1311 TFLOP/s
-    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 28},  // m1000n1000k2000_bcol: tc1_128x64_s8_g8 195 TFLOP/s
-    {4096, 4096, 4096, 4096, 512, 512, 1, 0, 0},  // m4096n4096k512_bcol: tc1_128x256_s4_g8 599 TFLOP/s
+    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 28},  // m1000n1000k2000_bcol: tc1_128x64_s8_g8 188 TFLOP/s
+    {4096, 4096, 4096, 4096, 512, 512, 1, 0, 0},  // m4096n4096k512_bcol: tc1_128x256_s4_g8 579 TFLOP/s
     {16, 16, 8192, 8192, 8192, 8192, 1, 0, 21},  // m16n8192k8192_bcol: swap_128x16_s8_sk 62 TFLOP/s
     {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 704 TFLOP/s
     {16384, 16384, 4096, 4096, 4096, 4096, 0, 1, 0},  // moe8_n4096_k4096: tc1_128x256_s4_g8 1228 TFLOP/s

@@ -289,9 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool ok = wait_phase(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
       if (pieces_possible) {
         // the piece path below syncs the four epilogue warps, so they must
-        // agree on leaving: a failed wait always raises the abort flag first
-        epilogue_bar();
-        if (*reinterpret_cast<volatile int*>(&ctl->abort)) break;
+        // agree on leaving: one reduced answer for all 128 threads
+        if (epilogue_bar_any(!ok || *reinterpret_cast<volatile int*>(&ctl->abort))) break;
       } else if (!__all_sync(0xffffffffu, ok)) {
         break;
       }
@@ -312,31 +311,55 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool finish = true;  // this block stores the tile
       const float* tile0 = nullptr;
       if (w.count > 1) {
-        // ---- one piece of a split tile: park the partial, the last piece sums
-        float* part = p.ws + (w.t * p.slot_stride + w.idx) * PART;
-#pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 16) {
-          uint32_t v[16];
-          tsrc.get<16>(cc, v);
-          put_partial16(part, row_local, cc, v);
-        }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&acce_bar[a]));  // the accumulator is free again
-        __threadfence();
+        // ---- one piece of a split tile.  The tile's counter holds arrivals
+        // in its low 16 bits and written partials in its high 16 bits.  The
+        // last piece to arrive waits for the others' partials and sums all
+        // pieces (its own straight from tensor memory); every other piece
+        // parks its partial and signals it.
         epilogue_bar();
         if (row_local == 0) {
           const unsigned old = atomicAdd(&p.counters[w.t], 1u);
-          ctl->last = (old == static_cast<unsigned>(w.count - 1)) ? 1 : 0;
+          ctl->last = ((old & 0xFFFFu) == static_cast<unsigned>(w.count - 1)) ? 1 : 0;
         }
         epilogue_bar();
         finish = ctl->last != 0;
-        if (finish) {
+        if (!finish) {
+          float* part = p.ws + (w.t * p.slot_stride + w.idx) * PART;
+#pragma unroll 1
+          for (int cc = 0; cc < BN; cc += 16) {
+            uint32_t v[16];
+            tsrc.get<16>(cc, v);
+            put_partial16(part, row_local, cc, v);
+          }
+          tc_fence_before();
+          mbar_arrive(smem_u32(&acce_bar[a]));  // the accumulator is free again
           __threadfence();
+          epilogue_bar();
+          if (row_local == 0) atomicAdd(&p.counters[w.t], 0x10000u);
+        } else {
+          bool gave_up = false;
+          if (row_local == 0) {
+            // every other piece has arrived, so each is writing its partial
+            // and will signal without waiting on anything: a bounded wait
+            const unsigned need = static_cast<unsigned>(w.count - 1);
+            const volatile unsigned* cnt = p.counters + w.t;
+            const uint64_t t0 = global_timer_ns();
+            while ((*cnt >> 16) < need) {
+              if (global_timer_ns() - t0 > p.timeout_ns) {
+                atomicCAS(p.status, 0u, kStatusTimeoutEpilogue);
+                *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+                gave_up = true;
+                break;
+              }
+            }
+            __threadfence();
+          }
+          if (epilogue_bar_any(gave_up)) break;
           tile0 = p.ws + w.t * p.slot_stride * PART;
         }
       }
       if (finish) {
-        const PartialSrc psrc{tile0, PART, w.count, row_local};
+        const PieceSumSrc psrc{tsrc, tile0, PART, w.count, w.idx, row_local};
         if constexpr (!SWAP) {
           const InT* bias_g = bias_t;
           if (TMA_EPI && p.tma_store) {
@@ -380,10 +403,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
         if (w.count > 1 && row_local == 0) p.counters[w.t] = 0u;  // ready for the next launch
-      }
-      if (w.count == 1) {
         tc_fence_before();
-        mbar_arrive(smem_u32(&acce_bar[a]));
+        mbar_arrive(smem_u32(&acce_bar[a]));  // this block's accumulator has been read
       }
     }
     // every TMA store has finished reading shared memory before the block

@@ -101,6 +101,21 @@ __device__ __forceinline__ void epilogue_bar() {
   asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
+// The same barrier, returning whether `pred` held in any of the 128 threads:
+// one answer for all of them, so the four warps always take the same branch.
+__device__ __forceinline__ bool epilogue_bar_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "barrier.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred))
+      : "memory");
+  return r != 0;
+}
+
 // One unit of work: K blocks [kb0, kb1) of output tile t, piece `idx` of
 // the `count` pieces that together cover the tile's K range.
 struct Work {
@@ -491,22 +506,32 @@ struct TmemSrc {
 };
 
 // A partial-tile sum as a source (the last piece of a split tile).
-struct PartialSrc {
+// The sum of a split tile's pieces, for the piece that finishes it: piece
+// `own` is this block's accumulator in tensor memory (`acc`), every other
+// piece s is the fp32 partial tile at tile0 + s * stride.  Columns cc ..
+// cc+W-1 of this thread's row are summed in piece order, so the result does
+// not depend on which piece finished last; all W/4 loads of one partial are
+// issued before any is used (one memory round trip per piece, not W/4).
+// Returned as raw fp32 bits.
+struct PieceSumSrc {
+  TmemSrc acc;
   const float* tile0;
   long long stride;
-  int count, row;
-  // Columns cc .. cc+W-1 of this thread's row summed over the `count` partial
-  // tiles `stride` floats apart, in piece order (so the result does not
-  // depend on which block finished last); returned as raw fp32 bits.  All W/4
-  // loads of one piece are issued before any is used, so a piece costs one
-  // memory round trip, not W/4.
+  int count, own, row;
   template <int W>
   __device__ __forceinline__ void get(int cc, uint32_t (&v)[W]) const {
     static_assert(W % 16 == 0, "whole 16-column groups");
     float f[W];
 #pragma unroll
     for (int j = 0; j < W; ++j) f[j] = 0.0f;
-    for (int s = 0; s < count; ++s) {
+    for (int s = 0; s < count; ++s) {  // warp-uniform
+      if (s == own) {
+        uint32_t t[W];
+        acc.get<W>(cc, t);
+#pragma unroll
+        for (int j = 0; j < W; ++j) f[j] += __uint_as_float(t[j]);
+        continue;
+      }
       const float4* q = reinterpret_cast<const float4*>(tile0 + s * stride);
       float4 t[W / 4];
 #pragma unroll
