@@ -64,7 +64,7 @@ static const Rule kRules[] = {
     {256, 256, 256, 256, 256, 256, 0, 0, 28},  // square256: tc1_128x64_s8_g8 3 TFLOP/s
     {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 28},  // m1024n1024k2048: tc1_128x64_s8_g8 209 TFLOP/s
     {2048, 2048, 2048, 2048, 2048, 2048, 0, 0, 0},  // square2048: tc1_128x256_s4_g8 672 TFLOP/s
-    {4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 11},  // square4096 (sustained): pair_256x256_s6_g16 1285 TFLOP/s
+    {4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 13},  // square4096: pair_256x512_s4_g16 1317 TFLOP/s
     {8192, 8192, 8192, 8192, 8192, 8192, 0, 0, 13},  // square8192 (sustained): pair_256x512_s4_g16 1311 TFLOP/s
     {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 28},  // m1000n1000k2000_bcol: tc1_128x64_s8_g8 188 TFLOP/s
     {4096, 4096, 4096, 4096, 512, 512, 1, 0, 0},  // m4096n4096k512_bcol: tc1_128x256_s4_g8 579 TFLOP/s
