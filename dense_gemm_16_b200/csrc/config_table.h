@@ -47,6 +47,8 @@ static const Config kConfigs[] = {
     {"tc1_128x64_s8_g8", kKindSingle, 64, 8, 8, 1, 2, 2},
     {"tc1_128x64_s8_g8_sk", kKindSingle, 64, 8, 8, -1, 2, 2},
     {"tc1_128x64_s8_g8_k2", kKindSingle, 64, 8, 8, 2, 2, 2},
+    {"csk_2x128x128_s4", kKindClusterSplitK, 128, 4, 8, 1, 2, 2},
+    {"csk_2x128x64_s6", kKindClusterSplitK, 64, 6, 8, 1, 2, 2},
 };
 static constexpr int kNumConfigs = static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0]));
 
@@ -62,11 +64,11 @@ struct Rule {
 // BEGIN RULES (written by the sweep)
 static const Rule kRules[] = {
     {256, 256, 256, 256, 256, 256, 0, 0, 28},  // square256: tc1_128x64_s8_g8 3 TFLOP/s
-    {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 28},  // m1024n1024k2048: tc1_128x64_s8_g8 209 TFLOP/s
+    {1024, 1024, 1024, 1024, 2048, 2048, 0, 0, 31},  // m1024n1024k2048: csk_2x128x128_s4 233 TFLOP/s
     {2048, 2048, 2048, 2048, 2048, 2048, 0, 0, 0},  // square2048: tc1_128x256_s4_g8 672 TFLOP/s
     {4096, 4096, 4096, 4096, 4096, 4096, 0, 0, 13},  // square4096: pair_256x512_s4_g16 1317 TFLOP/s
     {8192, 8192, 8192, 8192, 8192, 8192, 0, 0, 13},  // square8192 (sustained): pair_256x512_s4_g16 1311 TFLOP/s
-    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 28},  // m1000n1000k2000_bcol: tc1_128x64_s8_g8 188 TFLOP/s
+    {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 31},  // m1000n1000k2000_bcol: csk_2x128x128_s4 217 TFLOP/s
     {4096, 4096, 4096, 4096, 512, 512, 1, 0, 0},  // m4096n4096k512_bcol: tc1_128x256_s4_g8 579 TFLOP/s
     {16, 16, 8192, 8192, 8192, 8192, 1, 0, 21},  // m16n8192k8192_bcol: swap_128x16_s8_sk 62 TFLOP/s
     {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 704 TFLOP/s
@@ -88,6 +90,10 @@ inline int table_lookup(int M, int N, int K, bool b_col, bool grouped) {
   // the wide N fills the MMA rows; otherwise the widest tile that still puts
   // at least one tile on most SMs.
   if (!grouped && b_col && M <= 32) return M <= 16 ? 2 : 3;
+  // Few tiles and a long K loop: a CTA pair per 128 x 128 tile, each CTA
+  // one half of K, reduced in distributed shared memory
+  const long long tiles128 = static_cast<long long>((M + 127) / 128) * ((N + 127) / 128);
+  if (!grouped && tiles128 <= 64 && K >= 1024) return 31;
   const long long tiles256 = static_cast<long long>((M + 127) / 128) * ((N + 255) / 256);
   const long long pair_tiles = static_cast<long long>((M + 255) / 256) * ((N + 255) / 256);
   // CTA pairs halve the shared-memory operand traffic per MMA, which wins

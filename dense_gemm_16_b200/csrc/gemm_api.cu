@@ -316,6 +316,10 @@ KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool gro
     if (q_mn || grouped) return {nullptr, 0};  // needs column-major B
     return kernels_swap(c.bn, bf16, f32);
   }
+  if (c.kind == kKindClusterSplitK) {
+    if (grouped) return {nullptr, 0};
+    return kernels_csk(c.bn, q_mn, bf16, f32);
+  }
   if (c.kind == kKindGroupedSwap || c.kind == kKindGroupedSwapPair) {
     if (!grouped) return {nullptr, 0};
     return c.kind == kKindGroupedSwap ? kernels_gswap(c.bn, q_mn, bf16, f32)
@@ -361,6 +365,26 @@ int select_config(int M, int N, int K, unsigned epi, bool grouped) {
   const int forced = g_forced_config.load();
   if (forced >= 0) return forced;
   return table_lookup(M, N, K, (epi & GEMM_B_COL_MAJOR) != 0, grouped);
+}
+
+// The config a dense call runs: the table's (or the forced) choice, with two
+// substitutions when the choice came from the table: fp32 inputs run on the
+// single-CTA tf32 kernels only, and the CTA-pair split-K kernel, which needs
+// one SM pair per tile and two K blocks, gives way to 128 x 128 tiles when a
+// (batched) problem has more tiles than that.
+int dense_config(int batch, int M, int N, int K, unsigned epi, int dtype, const DeviceState* ds) {
+  int cid = select_config(M, N, K, epi, false);
+  if (cid < 0 || cid >= kNumConfigs || g_forced_config.load() >= 0) return cid;
+  if (in_tf32(dtype) && kConfigs[cid].kind != kKindSingle) {
+    const long long tiles256 = static_cast<long long>((M + 127) / 128) * ((N + 255) / 256);
+    return (N <= 128 || tiles256 < 96) ? 1 : 0;
+  }
+  if (kConfigs[cid].kind == kKindClusterSplitK) {
+    const long long tiles = static_cast<long long>(batch) * ((M + kBM - 1) / kBM) *
+                            ((N + kConfigs[cid].bn - 1) / kConfigs[cid].bn);
+    if (tiles > ds->num_sms / 2 || (K + kBK - 1) / kBK < 2) return 1;
+  }
+  return cid;
 }
 
 // One dense (optionally strided-batched) problem as the entry points take it.
@@ -441,6 +465,7 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   const bool f32 = out_bytes(d.dtype) == 4;
   const bool swap = cfg.kind == kKindSwap;
   const bool pair = cfg.kind == kKindPair;
+  const bool csk = cfg.kind == kKindClusterSplitK;
   const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false, tf32);
   const int ib = in_bytes(d.dtype);
   const uint32_t kbe = static_cast<uint32_t>(kb_elems(d.dtype));  // K per stage
@@ -539,7 +564,7 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   kp.slot_stride = 1;
   int grid_units = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms));
   const size_t counter_cap = fixed ? fixed->counter_slots : kCounterSlots;
-  if (!pair && splits != 1 && kp.num_kb >= 2 &&
+  if (!pair && !csk && splits != 1 && kp.num_kb >= 2 &&
       kp.num_tiles <= static_cast<long long>(counter_cap)) {
     if (splits > 1) {
       // split-K: every tile's K range in `splits` equal pieces
@@ -586,6 +611,11 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   if (pair) {
     const int pairs = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms / 2));
     return launch(k, 2 * pairs, stream, tp, tq, tc, kp, 2);
+  }
+  if (csk) {
+    // one CTA pair per tile, each CTA one half of the K blocks
+    if (kp.num_tiles > ds->num_sms / 2 || kp.num_kb < 2) return GEMM_ERR_UNSUPPORTED;
+    return launch(k, static_cast<int>(2 * kp.num_tiles), stream, tp, tq, tc, kp, 2);
   }
   return launch(k, grid_units, stream, tp, tq, tc, kp);
 }
@@ -648,13 +678,8 @@ int gemm_strided_batched(int batch, int M, int N, int K, const void* A, int64_t 
   rc = device_state(&ds);
   if (rc) return rc;
   if (K == 0) return fill_dispatch(d, stream);
-  int cid = select_config(M, N, K, epilogue, false);
+  const int cid = dense_config(batch, M, N, K, epilogue, dtype, ds);
   if (cid < 0 || cid >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
-  if (in_tf32(dtype) && kConfigs[cid].kind != kKindSingle && g_forced_config.load() < 0) {
-    // fp32 inputs run on the single-CTA tf32 kernels only
-    const long long tiles256 = static_cast<long long>((M + 127) / 128) * ((N + 255) / 256);
-    cid = (N <= 128 || tiles256 < 96) ? 1 : 0;
-  }
   return run_dense(ds, d, kConfigs[cid], kConfigs[cid].splits, nullptr, stream);
 }
 
@@ -696,7 +721,7 @@ int conv2d_im2col(int batch, int H, int W, int cin, int cout, int KH, int KW, in
   if (e != cudaSuccess) return cuda_fail(e);
   const DenseProblem d{1,     static_cast<int>(M), cout, static_cast<int>(K), A, lda, 0, w, cout,
                        0,     y, cout, 0, bias, 0, epilogue, dtype};
-  const int cid = select_config(d.M, d.N, d.K, epilogue, false);
+  const int cid = dense_config(1, d.M, d.N, d.K, epilogue, dtype, ds);
   if (cid < 0 || cid >= kNumConfigs) return GEMM_ERR_UNSUPPORTED;
   return run_dense(ds, d, kConfigs[cid], kConfigs[cid].splits, nullptr, stream);
 }

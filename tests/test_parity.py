@@ -73,7 +73,8 @@ def test_moe_grouped_sampled():
 
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("b_col", [False, True])
-@pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 12, 13, 23, 24, 28, 29, 30])
+@pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 12, 13, 23, 24, 28, 29, 30, 31,
+                                    32])
 def test_exact_integers(dtype, b_col, config):
     """Integer inputs in [-2, 2] with K <= 4096: every partial sum is an
     exact integer below 2^24, so the fp32 accumulator is exact in any order
@@ -144,7 +145,7 @@ def test_empty_m_or_n_is_a_noop():
     assert bool((g.ibuf.cpu() == g.sent).all())
 
 
-DENSE_CONFIGS = list(range(25)) + [28, 29, 30]  # 25..27 are grouped-only
+DENSE_CONFIGS = list(range(25)) + list(range(28, 33))  # 25..27 are grouped-only
 
 
 @pytest.mark.parametrize("config", DENSE_CONFIGS)
@@ -243,6 +244,82 @@ def test_trace_records_ordered_events_per_block(config):
     finally:
         dg.gemm_force_config(-1)
     assert torch.equal(C, C2)
+
+
+CSK = [31, 32]  # CTA-pair split-K reduced in distributed shared memory
+
+
+@pytest.mark.parametrize("config", CSK)
+@pytest.mark.parametrize("M,N,K,b_col", [
+    (74 * 128, 128, 256, False),  # 74 tiles of 128 x 128: every pair of SMs busy
+    (300, 200, 136, True),        # three K blocks: halves of 2 and 1
+    (1, 8, 128, False),           # one row, two K blocks
+])
+def test_pair_split_k_every_element(config, M, N, K, b_col):
+    assert dg.gemm_config_name(config).startswith("csk")
+    bn = 128 if config == 31 else 64
+    if ((M + 127) // 128) * ((N + bn - 1) // bn) > 74:
+        pytest.skip("more tiles than SM pairs")
+    gen = torch.Generator().manual_seed(M + N + K)
+    A = torch.randn(M, K, generator=gen).half()
+    B = torch.randn(*((N, K) if b_col else (K, N)), generator=gen).half()
+    bias = torch.randn(N, generator=gen).half()
+    ref = oracle.gemm(M, N, K, A, K, B, K if b_col else N, b_colmajor=b_col, bias=bias,
+                      relu=True, dtype="f16", threads=THREADS)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        g = run_gemm(A.cuda(), B.cuda(), bias.cuda(), M, N, K, b_col=b_col, relu=True)
+    finally:
+        dg.gemm_force_config(-1)
+    compare(g.matrix().double().cpu().numpy(), ref, 2, "pair split-K")
+    g.check_canaries()
+
+
+def test_table_choice_of_pair_split_k_and_its_batched_fallback():
+    # 512 x 512 x 2048 matches no rule: the heuristic takes the pair split-K
+    # kernel; 1024 x 1024 x 2048 in a batch of 2 has 128 tiles, more than the
+    # SM pairs, so the batched call runs 128 x 128 tiles instead
+    assert dg.gemm_config_name(dg.gemm_select_config(512, 512, 2048, dg.GEMM_F16, 0)) \
+        .startswith("csk")
+    gen = torch.Generator().manual_seed(31)
+    A = torch.randn(512, 2048, generator=gen).half()
+    B = torch.randn(2048, 512, generator=gen).half()
+    ref = oracle.gemm(512, 512, 2048, A, 2048, B, 512, dtype="f16", threads=THREADS)
+    g = run_gemm(A.cuda(), B.cuda(), None, 512, 512, 2048)
+    compare(g.matrix().double().cpu().numpy(), ref, 2, "heuristic pair split-K")
+    g.check_canaries()
+    M = N = 1024
+    K = 2048
+    A2 = torch.randn(2, M, K, generator=gen).half()
+    B2 = torch.randn(2, K, N, generator=gen).half()
+    C2 = torch.empty(2, M, N, dtype=torch.half, device="cuda")
+    rc = dg.gemm_strided_batched(2, M, N, K, A2.cuda(), K, M * K, B2.cuda(), N, K * N, C2, N,
+                                 M * N, None, 0, 0, dg.GEMM_F16)
+    assert rc == 0, dg.gemm_status_string(rc)
+    torch.cuda.synchronize()
+    assert dg.gemm_device_status() == 0
+    for b in range(2):
+        r, c = workloads.sample_indices(M, N, n=512, seed=b)
+        ref = oracle.gemm_at(M, N, K, A2[b], K, B2[b], N, r, c, dtype="f16", threads=THREADS)
+        compare(C2[b].double().cpu().numpy()[r, c], ref, 2, f"batched fallback {b}")
+
+
+@pytest.mark.parametrize("config", CSK)
+def test_pair_split_k_rejects_what_it_cannot_split(config):
+    # more tiles than SM pairs, or a single K block: UNSUPPORTED, nothing written
+    A = torch.ones(4096, 256, dtype=torch.half, device="cuda")
+    B = torch.ones(256, 4096, dtype=torch.half, device="cuda")
+    C = torch.zeros(4096, 4096, dtype=torch.half, device="cuda")
+    assert dg.gemm_force_config(config) == 0
+    try:
+        assert dg.gemm(4096, 4096, 256, A, 256, B, 4096, C, 4096, None, 0,
+                       dg.GEMM_F16) == dg.GEMM_ERR_UNSUPPORTED
+        assert dg.gemm(128, 128, 64, A, 256, B, 4096, C, 4096, None, 0,
+                       dg.GEMM_F16) == dg.GEMM_ERR_UNSUPPORTED
+    finally:
+        dg.gemm_force_config(-1)
+    torch.cuda.synchronize()
+    assert int(C.abs().sum()) == 0
 
 
 def test_runs_on_a_side_stream():
