@@ -20,17 +20,31 @@
 
 namespace dg16 {
 
+constexpr int kCskChunk = 32;  // columns per transfer chunk (one barrier each)
+
 // Where rank 1's partial lands in rank 0: [BN/4][128 rows][4] fp32, so the
-// 32 lanes of a warp (32 consecutive rows) touch 512 contiguous bytes.
+// 32 lanes of a warp (32 consecutive rows) touch 512 contiguous bytes.  It
+// arrives in chunks of kCskChunk columns, each with its own barrier; rank 0
+// loads its own accumulator columns first and waits for the matching chunks
+// only then, so its epilogue overlaps the rest of the transfer.
 template <int BN>
 struct CskRecvSrc {
   TmemSrc acc;     // rank 0's accumulator
   uint32_t recv;   // shared-memory address of the received partial
+  uint32_t bar0;   // shared-memory address of the first chunk's barrier
   int row;
+  SharedCtl* ctl;
+  const KParams* p;
   template <int W>
   __device__ __forceinline__ void get(int cc, uint32_t (&v)[W]) const {
+    static_assert(W % kCskChunk == 0 || kCskChunk % W == 0, "whole chunks");
     uint32_t t[W];
     acc.get<W>(cc, t);
+    // a chunk that never arrives leaves its values undefined; the bounded
+    // wait has then recorded the error in the status word
+    for (int c = cc / kCskChunk; c * kCskChunk < cc + W; ++c)
+      (void)wait_phase<true>(bar0 + static_cast<uint32_t>(c) * 8u, 0, ctl, *p,
+                             kStatusTimeoutEpilogue);
 #pragma unroll
     for (int j = 0; j < W / 4; ++j) {
       const uint32_t a =
@@ -69,12 +83,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sStage = sQ + STAGES * Q_BYTES;   // epilogue staging (rank 0)
   uint8_t* sRecv = sStage + kEpiStageBytes;  // rank 1's partial (rank 0)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRecv + RECV_BYTES);
+  constexpr int NCHUNK = BN / kCskChunk;
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* accf_bar = bars + 2 * STAGES;
-  uint64_t* recv_bar = bars + 2 * STAGES + 1;
-  uint64_t* drain_bar = bars + 2 * STAGES + 2;
-  SharedCtl* ctl = reinterpret_cast<SharedCtl*>(bars + 2 * STAGES + 3);
+  uint64_t* drain_bar = bars + 2 * STAGES + 1;
+  uint64_t* recv_bar = bars + 2 * STAGES + 2;  // NCHUNK barriers
+  SharedCtl* ctl = reinterpret_cast<SharedCtl*>(bars + 2 * STAGES + 2 + NCHUNK);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -87,7 +102,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&empty_bar[s]), 1);
     }
     mbar_init(smem_u32(accf_bar), 1);
-    mbar_init(smem_u32(recv_bar), 4 * 32);  // every epilogue thread of rank 1
+    for (int c = 0; c < NCHUNK; ++c)
+      mbar_init(smem_u32(&recv_bar[c]), 4 * 32);  // every epilogue thread of rank 1
     mbar_init(smem_u32(drain_bar), 1);
     ctl->abort = 0;
     fence_barrier_init();
@@ -198,29 +214,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         // fp32 accumulator -> rank 0's receive buffer, then one arrival per
         // thread (release at cluster scope: the stores are visible first)
         const uint32_t recv0 = map_shared_rank(smem_u32(sRecv), 0);
+        const uint32_t rbar0 = map_shared_rank(smem_u32(&recv_bar[0]), 0);
 #pragma unroll 1
-        for (int cc = 0; cc < BN; cc += 16) {
-          uint32_t v[16];
-          tsrc.get<16>(cc, v);
+        for (int cc = 0; cc < BN; cc += kCskChunk) {
+          uint32_t v[kCskChunk];
+          tsrc.get<kCskChunk>(cc, v);
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
+          for (int j = 0; j < kCskChunk / 4; ++j) {
             const uint32_t a =
                 recv0 + static_cast<uint32_t>(((cc / 4 + j) * kBM + row_local) * 16);
             asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
                          "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
                          : "memory");
           }
+          mbar_arrive_cluster(rbar0 + static_cast<uint32_t>(cc / kCskChunk) * 8u);
         }
-        mbar_arrive_cluster(map_shared_rank(smem_u32(recv_bar), 0));
       } else {
-        // rank 1's half has arrived: sum in rank order, bias, ReLU, store
-        const bool got = wait_phase<true>(smem_u32(recv_bar), 0, ctl, p, kStatusTimeoutEpilogue);
-        if (__all_sync(0xffffffffu, got)) {
+        // sum in rank order as rank 1's chunks arrive, bias, ReLU, store
+        {
           const InT* bias = (p.epi & 1) ? reinterpret_cast<const InT*>(p.bias) +
                                               static_cast<long long>(c.group) * p.stride_bias
                                         : nullptr;
           const bool relu = (p.epi & 2) != 0;
-          const CskRecvSrc<BN> src{tsrc, smem_u32(sRecv), row_local};
+          const CskRecvSrc<BN> src{tsrc, smem_u32(sRecv), smem_u32(&recv_bar[0]), row_local, ctl, &p};
           const int q0 = c.q0 * BN;
           if (p.tma_store) {
             uint32_t stores = 0;
@@ -252,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int STAGES>
 constexpr int gemm_csk_smem_bytes() {
   return 1024 + STAGES * (kBM * 128 + BN * 128) + static_cast<int>(kEpiStageBytes) +
-         kBM * BN * 4 + (2 * STAGES + 3) * 8 + static_cast<int>(sizeof(SharedCtl));
+         kBM * BN * 4 + (2 * STAGES + 2 + BN / kCskChunk) * 8 + static_cast<int>(sizeof(SharedCtl));
 }
 
 }  // namespace dg16
