@@ -59,25 +59,34 @@ def _peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def _source_sha() -> str:
+# Sources every launch depends on (host path, shared device code, the table).
+_COMMON_SOURCES = ("ptx.cuh", "kernel_common.cuh", "raster.h", "dispatch.h", "config_table.h",
+                   "gemm_api.cu")
+
+
+def _source_sha(files=None) -> str:
+    """Hash of the named csrc files (all of them when None)."""
+    csrc = os.path.join(ROOT, "dense_gemm_16_b200", "csrc")
+    names = sorted(files) if files else sorted(os.listdir(csrc))
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "dense_gemm_16_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode())
+    for name in names:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def _traffic(workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the same kernel sources and workload; else None."""
+    on this workload with the same sources of the kernel that runs it (the
+    entry lists them: the common files plus that kernel's own); else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
     entry = d.get(workload)
-    if not entry or entry.get("source_sha") != _source_sha():
+    if not entry or entry.get("source_sha") != _source_sha(entry.get("sources")):
         return None
     return entry.get("dram_bytes_per_launch")
 
