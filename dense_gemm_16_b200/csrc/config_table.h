@@ -49,6 +49,7 @@ static const Config kConfigs[] = {
     {"tc1_128x64_s8_g8_k2", kKindSingle, 64, 8, 8, 2, 2, 2},
     {"csk_2x128x128_s4", kKindClusterSplitK, 128, 4, 8, 1, 2, 2},
     {"csk_2x128x64_s6", kKindClusterSplitK, 64, 6, 8, 1, 2, 2},
+    {"cskswap_2x128x16_s10", kKindClusterSplitKSwap, 16, 10, 1, 1, 1, 2},
 };
 static constexpr int kNumConfigs = static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0]));
 

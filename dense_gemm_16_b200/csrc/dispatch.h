@@ -22,6 +22,7 @@ enum ConfigKind : int {
   kKindGroupedSwapPair = 4,  // the same with a CTA pair per 256 columns x <= bn rows
   kKindClusterSplitK = 5,    // dense, tiles <= SMs / 2: a CTA pair per 128 x bn tile,
                              // one half of K each, reduced in distributed shared memory
+  kKindClusterSplitKSwap = 6,  // the same for skinny problems, operands swapped (C^T)
 };
 
 struct Config {
@@ -46,6 +47,7 @@ KernelEntry kernels_tf32(int bn, bool q_mn);
 KernelEntry kernels_gswap(int tok, bool p_mn, bool bf16, bool out_f32);
 KernelEntry kernels_gswap2(int tok, bool p_mn, bool bf16, bool out_f32);
 KernelEntry kernels_csk(int bn, bool q_mn, bool bf16, bool out_f32);
+KernelEntry kernels_csk_swap(int bn, bool bf16, bool out_f32);
 
 // NHWC im2col gather (im2col.cu): A[m][k] for M = batch*OH*OW, K = KH*KW*cin.
 cudaError_t launch_im2col(const void* x, void* A, long long lda, int batch, int H, int W, int cin,

@@ -320,6 +320,10 @@ KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool gro
     if (grouped) return {nullptr, 0};
     return kernels_csk(c.bn, q_mn, bf16, f32);
   }
+  if (c.kind == kKindClusterSplitKSwap) {
+    if (q_mn || grouped) return {nullptr, 0};  // needs column-major B
+    return kernels_csk_swap(c.bn, bf16, f32);
+  }
   if (c.kind == kKindGroupedSwap || c.kind == kKindGroupedSwapPair) {
     if (!grouped) return {nullptr, 0};
     return c.kind == kKindGroupedSwap ? kernels_gswap(c.bn, q_mn, bf16, f32)
@@ -379,10 +383,13 @@ int dense_config(int batch, int M, int N, int K, unsigned epi, int dtype, const 
     const long long tiles256 = static_cast<long long>((M + 127) / 128) * ((N + 255) / 256);
     return (N <= 128 || tiles256 < 96) ? 1 : 0;
   }
-  if (kConfigs[cid].kind == kKindClusterSplitK) {
-    const long long tiles = static_cast<long long>(batch) * ((M + kBM - 1) / kBM) *
-                            ((N + kConfigs[cid].bn - 1) / kConfigs[cid].bn);
-    if (tiles > ds->num_sms / 2 || (K + kBK - 1) / kBK < 2) return 1;
+  const int kind = kConfigs[cid].kind;
+  if (kind == kKindClusterSplitK || kind == kKindClusterSplitKSwap) {
+    const bool sw = kind == kKindClusterSplitKSwap;
+    const int rows = sw ? N : M, cols = sw ? M : N;  // MMA rows / MMA-N of the tiles
+    const long long tiles = static_cast<long long>(batch) * ((rows + kBM - 1) / kBM) *
+                            ((cols + kConfigs[cid].bn - 1) / kConfigs[cid].bn);
+    if (tiles > ds->num_sms / 2 || (K + kBK - 1) / kBK < 2) return sw ? 21 : 1;
   }
   return cid;
 }
@@ -463,9 +470,9 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   const bool bf16 = in_bf16(d.dtype);
   const bool tf32 = in_tf32(d.dtype);
   const bool f32 = out_bytes(d.dtype) == 4;
-  const bool swap = cfg.kind == kKindSwap;
+  const bool swap = cfg.kind == kKindSwap || cfg.kind == kKindClusterSplitKSwap;
   const bool pair = cfg.kind == kKindPair;
-  const bool csk = cfg.kind == kKindClusterSplitK;
+  const bool csk = cfg.kind == kKindClusterSplitK || cfg.kind == kKindClusterSplitKSwap;
   const KernelEntry k = kernel_for(cfg, swap ? false : !bcol, bf16, f32, false, tf32);
   const int ib = in_bytes(d.dtype);
   const uint32_t kbe = static_cast<uint32_t>(kb_elems(d.dtype));  // K per stage

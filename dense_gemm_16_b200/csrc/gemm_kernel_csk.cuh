@@ -13,7 +13,9 @@
 // SM-to-SM transfer of 64 KB.
 //
 // One tile per pair: the launch has exactly two CTAs per tile, so it is used
-// only where tiles <= SMs / 2.  No load is multicast.
+// only where tiles <= SMs / 2.  No load is multicast.  The swapped form (the
+// skinny 16 x 8192 x 8192 problem: 64 tiles of 128 columns of B) streams
+// each half of B once and hands over 8 KB per tile.
 #pragma once
 
 #include "kernel_common.cuh"
@@ -27,7 +29,7 @@ constexpr int kCskChunk = 32;  // columns per transfer chunk (one barrier each)
 // arrives in chunks of kCskChunk columns, each with its own barrier; rank 0
 // loads its own accumulator columns first and waits for the matching chunks
 // only then, so its epilogue overlaps the rest of the transfer.
-template <int BN>
+template <int BN, int CH>
 struct CskRecvSrc {
   TmemSrc acc;     // rank 0's accumulator
   uint32_t recv;   // shared-memory address of the received partial
@@ -37,12 +39,12 @@ struct CskRecvSrc {
   const KParams* p;
   template <int W>
   __device__ __forceinline__ void get(int cc, uint32_t (&v)[W]) const {
-    static_assert(W % kCskChunk == 0 || kCskChunk % W == 0, "whole chunks");
+    static_assert(W % CH == 0 || CH % W == 0, "whole chunks");
     uint32_t t[W];
     acc.get<W>(cc, t);
     // a chunk that never arrives leaves its values undefined; the bounded
     // wait has then recorded the error in the status word
-    for (int c = cc / kCskChunk; c * kCskChunk < cc + W; ++c)
+    for (int c = cc / CH; c * CH < cc + W; ++c)
       (void)wait_phase<true>(bar0 + static_cast<uint32_t>(c) * 8u, 0, ctl, *p,
                              kStatusTimeoutEpilogue);
 #pragma unroll
@@ -62,12 +64,17 @@ struct CskRecvSrc {
 };
 
 //   BN, STAGES, Q_MN, IN_BF16, OutT as in gemm_tc_kernel (dense tiles only)
-template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT>
+//   SWAP    skinny problems: P = B stored N x K, Q = A, the accumulator holds
+//           C^T (N on the 128 MMA rows, BN = 16 or 32 rows of A on MMA-N)
+template <int BN, int STAGES, bool Q_MN, bool IN_BF16, typename OutT, bool SWAP = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_csk_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ KParams p) {
   using InT = typename std::conditional<IN_BF16, __nv_bfloat16, __half>::type;
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN of 64..256, whole 64-column chunks");
+  static_assert(SWAP ? ((BN == 16 || BN == 32) && !Q_MN)
+                     : (BN % 64 == 0 && BN >= 64 && BN <= 256),
+                "BN of 64..256 in whole 64-column chunks; swapped: 16 or 32, K-major A");
+  constexpr int CH = BN < kCskChunk ? BN : kCskChunk;  // columns per transfer chunk
   constexpr uint32_t P_BYTES = kBM * 128;
   constexpr uint32_t Q_BYTES = BN * 128;
   constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
@@ -83,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sStage = sQ + STAGES * Q_BYTES;   // epilogue staging (rank 0)
   uint8_t* sRecv = sStage + kEpiStageBytes;  // rank 1's partial (rank 0)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sRecv + RECV_BYTES);
-  constexpr int NCHUNK = BN / kCskChunk;
+  constexpr int NCHUNK = BN / CH;
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* accf_bar = bars + 2 * STAGES;
@@ -216,18 +223,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t recv0 = map_shared_rank(smem_u32(sRecv), 0);
         const uint32_t rbar0 = map_shared_rank(smem_u32(&recv_bar[0]), 0);
 #pragma unroll 1
-        for (int cc = 0; cc < BN; cc += kCskChunk) {
-          uint32_t v[kCskChunk];
-          tsrc.get<kCskChunk>(cc, v);
+        for (int cc = 0; cc < BN; cc += CH) {
+          uint32_t v[CH];
+          tsrc.get<CH>(cc, v);
 #pragma unroll
-          for (int j = 0; j < kCskChunk / 4; ++j) {
+          for (int j = 0; j < CH / 4; ++j) {
             const uint32_t a =
                 recv0 + static_cast<uint32_t>(((cc / 4 + j) * kBM + row_local) * 16);
             asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
                          "r"(v[4 * j]), "r"(v[4 * j + 1]), "r"(v[4 * j + 2]), "r"(v[4 * j + 3])
                          : "memory");
           }
-          mbar_arrive_cluster(rbar0 + static_cast<uint32_t>(cc / kCskChunk) * 8u);
+          mbar_arrive_cluster(rbar0 + static_cast<uint32_t>(cc / CH) * 8u);
         }
       } else {
         // sum in rank order as rank 1's chunks arrive, bias, ReLU, store
@@ -236,9 +243,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                                               static_cast<long long>(c.group) * p.stride_bias
                                         : nullptr;
           const bool relu = (p.epi & 2) != 0;
-          const CskRecvSrc<BN> src{tsrc, smem_u32(sRecv), smem_u32(&recv_bar[0]), row_local, ctl, &p};
+          const CskRecvSrc<BN, CH> src{tsrc,     smem_u32(sRecv), smem_u32(&recv_bar[0]),
+                                       row_local, ctl,      &p};
           const int q0 = c.q0 * BN;
-          if (p.tma_store) {
+          if constexpr (SWAP) {
+            // accumulator row = output column n; its columns are output rows
+            // q0 .. q0+BN
+            const int n = c.p0 + row_local;
+            const bool col_ok = n < p.N;
+            const float b = (bias != nullptr && col_ok) ? to_f32<InT>(bias[n]) : 0.0f;
+            OutT* const C =
+                reinterpret_cast<OutT*>(p.C) + static_cast<long long>(c.group) * p.stride_c;
+#pragma unroll 1
+            for (int cc = 0; cc < BN; cc += 16) {
+              const int row0 = q0 + cc;
+              if (row0 >= p.M) break;  // warp-uniform
+              uint32_t v[16];
+              src.template get<16>(cc, v);
+              if (col_ok) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  if (row0 + j < p.M) {
+                    float x = __uint_as_float(v[j]) + b;
+                    if (relu) x = fmaxf(x, 0.0f);
+                    C[static_cast<long long>(row0 + j) * p.ldc + n] = from_f32<OutT>(x);
+                  }
+                }
+              }
+            }
+          } else if (p.tma_store) {
             uint32_t stores = 0;
             const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>(warp - 2) * 8192u;
             store_tma_from<BN, InT, OutT>(src, c.p0 + quad * 32, q0, c.group, p, bias, relu,
@@ -268,7 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int STAGES>
 constexpr int gemm_csk_smem_bytes() {
   return 1024 + STAGES * (kBM * 128 + BN * 128) + static_cast<int>(kEpiStageBytes) +
-         kBM * BN * 4 + (2 * STAGES + 2 + BN / kCskChunk) * 8 + static_cast<int>(sizeof(SharedCtl));
+         kBM * BN * 4 + (2 * STAGES + 2 + BN / (BN < kCskChunk ? BN : kCskChunk)) * 8 +
+         static_cast<int>(sizeof(SharedCtl));
 }
 
 }  // namespace dg16

@@ -6,11 +6,11 @@
 
 namespace dg16 {
 
-template <int BN, int S, bool Q_MN, bool BF16, bool F32>
+template <int BN, int S, bool Q_MN, bool BF16, bool F32, bool SWAP = false>
 static KernelEntry entry_csk() {
   using In = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   using Out = typename std::conditional<F32, float, In>::type;
-  return {reinterpret_cast<const void*>(&gemm_csk_kernel<BN, S, Q_MN, BF16, Out>),
+  return {reinterpret_cast<const void*>(&gemm_csk_kernel<BN, S, Q_MN, BF16, Out, SWAP>),
           gemm_csk_smem_bytes<BN, S>()};
 }
 
@@ -35,6 +35,19 @@ KernelEntry kernels_csk(int bn, bool q_mn, bool bf16, bool out_f32) {
   if (bn == 128) return pick_csk<128, 4>(q_mn, bf16, out_f32);
   if (bn == 64) return pick_csk<64, 6>(q_mn, bf16, out_f32);
   return {nullptr, 0};
+}
+
+// Swapped (skinny, column-major B): 128 columns of B x 16 rows of A per
+// tile, a 10-stage ring of 18 KB.
+KernelEntry kernels_csk_swap(int bn, bool bf16, bool out_f32) {
+  if (bn != 16) return {nullptr, 0};
+  const int key = (bf16 ? 2 : 0) | (out_f32 ? 1 : 0);
+  switch (key) {
+    case 0: return entry_csk<16, 10, false, false, false, true>();
+    case 1: return entry_csk<16, 10, false, false, true, true>();
+    case 2: return entry_csk<16, 10, false, true, false, true>();
+    default: return entry_csk<16, 10, false, true, true, true>();
+  }
 }
 
 }  // namespace dg16

@@ -145,7 +145,7 @@ def test_empty_m_or_n_is_a_noop():
     assert bool((g.ibuf.cpu() == g.sent).all())
 
 
-DENSE_CONFIGS = list(range(25)) + list(range(28, 33))  # 25..27 are grouped-only
+DENSE_CONFIGS = list(range(25)) + list(range(28, 34))  # 25..27 are grouped-only
 
 
 @pytest.mark.parametrize("config", DENSE_CONFIGS)
@@ -154,7 +154,7 @@ DENSE_CONFIGS = list(range(25)) + list(range(28, 33))  # 25..27 are grouped-only
 def test_every_config_on_ragged_problem(config, dtype, out_f32):
     assert config < dg.gemm_num_configs()
     name = dg.gemm_config_name(config)
-    swap = name.startswith("swap")
+    swap = name.startswith(("swap", "cskswap"))
     M, N, K = (29 if swap else 333), 712, 328
     gen = torch.Generator().manual_seed(1000 + config)
     A = torch.randn(M, K, generator=gen).to(dtype)
@@ -302,6 +302,26 @@ def test_table_choice_of_pair_split_k_and_its_batched_fallback():
         r, c = workloads.sample_indices(M, N, n=512, seed=b)
         ref = oracle.gemm_at(M, N, K, A2[b], K, B2[b], N, r, c, dtype="f16", threads=THREADS)
         compare(C2[b].double().cpu().numpy()[r, c], ref, 2, f"batched fallback {b}")
+
+
+@pytest.mark.parametrize("M,N,K", [(16, 8192, 2048), (29, 712, 328), (1, 1000, 136)])
+def test_pair_split_k_swapped_every_element(M, N, K):
+    # skinny problems: B column-major, C^T in the accumulators, 8 KB handed over
+    config = 33
+    assert dg.gemm_config_name(config).startswith("cskswap")
+    gen = torch.Generator().manual_seed(M * 7 + K)
+    A = torch.randn(M, K, generator=gen).half()
+    B = torch.randn(N, K, generator=gen).half()
+    bias = torch.randn(N, generator=gen).half()
+    ref = oracle.gemm(M, N, K, A, K, B, K, b_colmajor=True, bias=bias, relu=True, dtype="f16",
+                      threads=THREADS)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        g = run_gemm(A.cuda(), B.cuda(), bias.cuda(), M, N, K, b_col=True, relu=True)
+    finally:
+        dg.gemm_force_config(-1)
+    compare(g.matrix().double().cpu().numpy(), ref, 2, "swapped pair split-K")
+    g.check_canaries()
 
 
 @pytest.mark.parametrize("config", CSK)
