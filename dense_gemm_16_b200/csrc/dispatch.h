@@ -31,7 +31,8 @@ struct Config {
   int bn;       // MMA N (Q rows per tile)
   int stages;   // operand ring depth
   int group_m;  // raster band height
-  int splits;   // split-K factor (1 = whole K per tile; -1 = stream-K)
+  int splits;   // split-K factor (1 = whole K per tile; -1 = stream-K; -2 = hybrid
+                //  stream-K over the last waves' tiles)
   int pol_p;    // L2 eviction policy of the 128-row operand's copies (kPolicy*)
   int pol_q;    // ... and of the BN-row operand's copies
 };

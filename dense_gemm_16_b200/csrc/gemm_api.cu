@@ -581,6 +581,12 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
       kp.splits = (kp.num_kb + per - 1) / per;  // no empty K range
       kp.slot_stride = kp.splits;
       grid_units = static_cast<int>(std::min<long long>(kp.num_tiles * kp.splits, ds->num_sms));
+    } else if (splits == -2) {
+      // hybrid: stream-K over the last waves' tiles, whole tiles before
+      // them; the kernel derives the split from the tile count and grid
+      kp.work_mode = 3;
+      kp.sk_width = 1;
+      grid_units = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms));
     } else {
       // stream-K: every block gets an equal share of the (tile, K block)
       // iterations, cut at tile edges
@@ -593,8 +599,10 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
     if (kp.work_mode == 1 && kp.splits == 1) kp.work_mode = 0;
   }
   if (kp.work_mode != 0) {
-    const size_t partial =
-        static_cast<size_t>(kp.num_tiles) * kp.slot_stride * kBM * cfg.bn * 4;
+    // split-K: slot_stride slots per tile; stream-K: two per block
+    const size_t slots = kp.work_mode >= 2 ? 2 * static_cast<size_t>(grid_units)
+                                           : static_cast<size_t>(kp.num_tiles) * kp.slot_stride;
+    const size_t partial = slots * kBM * cfg.bn * 4;
     if (fixed) {
       if (partial > fixed->partial_bytes) return GEMM_ERR_UNSUPPORTED;  // beyond the scratch
       kp.ws = fixed->ws;
@@ -914,12 +922,25 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
   kp.splits = 1;
   kp.kb_per_split = kp.num_kb;
   kp.slot_stride = 1;
+  kp.sk_width = 1;
   // upper bound on tiles: each group adds at most one partial row block
   const long long nq = (N + cfg.bn - 1) / cfg.bn;
   const long long max_tiles = (static_cast<long long>(total_rows) / kBM + num_groups) * nq;
   CUtensorMap tc;
   std::memset(&tc, 0, sizeof(tc));  // grouped tiles store from registers
   const int grid = static_cast<int>(std::min<long long>(max_tiles, ds->num_sms));
+  if (cfg.splits < 0 && kp.num_kb >= 2 && max_tiles <= static_cast<long long>(kCounterSlots)) {
+    // stream-K (-1) or the hybrid (-2) over the (tile, K block) space; the
+    // kernel derives the width from the tile count it computes from the
+    // group sizes
+    kp.work_mode = cfg.splits == -2 ? 3 : 2;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    rc = stream_workspace(dev, stream, 2 * static_cast<size_t>(grid) * kBM * cfg.bn * 4, &kp.ws,
+                          &kp.counters);
+    if (rc) return rc;
+  }
   return launch(k, grid, stream, tp, tq, tc, kp);
 }
 

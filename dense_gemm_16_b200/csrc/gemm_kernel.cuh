@@ -153,6 +153,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   long long num_tiles = p.num_tiles;
   if constexpr (GROUPED) num_tiles = gt->tile_start[p.num_groups];
+  // grouped stream-K: the width follows from the tile count computed above
+  // (the host cannot know it); the hybrid mode derives its split here for
+  // both kinds.  The same values in every role.
+  long long sk_width = 0, sk_tiles = 0;
+  if (p.work_mode == 3)
+    hybrid_split(num_tiles, p.num_kb, &sk_tiles, &sk_width);
+  else if (GROUPED && p.work_mode == 2)
+    sk_width =
+        max(1ll, (num_tiles * p.num_kb + gridDim.x - 1) / static_cast<long long>(gridDim.x));
   const int num_q_blocks = GROUPED ? (p.N + BN - 1) / BN : p.num_q;
 
   if (warp == 0) {
@@ -163,7 +172,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       int gcur = 0;
       bool ok = true;
-      WorkIter wi(p, num_tiles);
+      WorkIter wi(p, num_tiles, sk_width, sk_tiles);
       Work w;
       while (ok && wi.next(p, w)) {
         const TileCoord c = tile_coord<GROUPED>(w.t, p, num_q_blocks, gt, gcur);
@@ -209,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, local = 0;
       int gcur = 0;
       bool ok = true;
-      WorkIter wi(p, num_tiles);
+      WorkIter wi(p, num_tiles, sk_width, sk_tiles);
       Work w;
       for (; ok && wi.next(p, w); ++local) {
         const TileCoord c = tile_coord<GROUPED>(w.t, p, num_q_blocks, gt, gcur);
@@ -277,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool relu = (p.epi & 2) != 0;
     const bool pieces_possible = p.work_mode != 0;  // uniform for the launch
     constexpr long long PART = static_cast<long long>(kBM) * BN;  // floats per partial tile
-    WorkIter wi(p, num_tiles);
+    WorkIter wi(p, num_tiles, sk_width, sk_tiles);
     Work w;
     for (; wi.next(p, w); ++local) {
       const TileCoord c = tile_coord<GROUPED>(w.t, p, num_q_blocks, gt, gcur);
@@ -309,7 +318,6 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * ACC_COLS;
       const TmemSrc tsrc{taddr, min(NACC, 4 * (w.kb1 - w.kb0)), BN};
       bool finish = true;  // this block stores the tile
-      const float* tile0 = nullptr;
       if (w.count > 1) {
         // ---- one piece of a split tile.  The tile's counter holds arrivals
         // in its low 16 bits and written partials in its high 16 bits.  The
@@ -324,7 +332,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         epilogue_bar();
         finish = ctl->last != 0;
         if (!finish) {
-          float* part = p.ws + (w.t * p.slot_stride + w.idx) * PART;
+          float* part =
+              p.ws + piece_slot(p, w.t, w.idx, static_cast<long long>(blockIdx.x) - w.idx) * PART;
 #pragma unroll 1
           for (int cc = 0; cc < BN; cc += 16) {
             uint32_t v[16];
@@ -355,11 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             __threadfence();
           }
           if (epilogue_bar_any(gave_up)) break;
-          tile0 = p.ws + w.t * p.slot_stride * PART;
         }
       }
       if (finish) {
-        const PieceSumSrc psrc{tsrc, tile0, PART, w.count, w.idx, row_local};
+        const PieceSumSrc psrc{tsrc,    &p,      w.t,   static_cast<long long>(blockIdx.x) - w.idx,
+                               PART,    w.count, w.idx, row_local};
         if constexpr (!SWAP) {
           const InT* bias_g = bias_t;
           if (TMA_EPI && p.tma_store) {

@@ -50,6 +50,8 @@ struct KParams {
   //                kb_per_split blocks
   //   work_mode 2  stream-K: block b takes iterations [b*sk_width,
   //                (b+1)*sk_width) of the (tile, K block) space
+  //   work_mode 3  hybrid: stream-K over the tiles of the last waves, whole
+  //                tiles for the rest (see WorkIter)
   // A tile computed in several pieces parks fp32 partial tiles in `ws`
   // (slot tile*slot_stride + piece) and the last piece to finish sums them
   // in piece order and runs the epilogue.
@@ -126,14 +128,34 @@ struct Work {
 
 // The sequence of work units one block processes, in the same order for the
 // producer, the MMA issuer and the epilogue.
+//   work_mode 0: whole tiles t = block, block + grid, ...
+//   work_mode 1: split-K units (tile, split), strided the same way
+//   work_mode 2: stream-K: block b takes iterations [b*W, (b+1)*W) of the
+//                (tile, K block) space, W = sk_width
+//   work_mode 3: hybrid: stream-K over the first sk_tiles tiles (the tiles
+//                that do not fill whole waves, plus one wave), then whole
+//                tiles sk_tiles + block, + grid, ... for the rest, so most
+//                of the work keeps the raster's L2 locality
 struct WorkIter {
   long long cursor, end, step;
-  __device__ __forceinline__ WorkIter(const KParams& p, long long num_tiles) {
-    if (p.work_mode == 2) {
-      const long long total = num_tiles * p.num_kb;
-      cursor = static_cast<long long>(blockIdx.x) * p.sk_width;
-      end = min(total, cursor + p.sk_width);
+  long long sk_width;  // stream-K: iterations per block
+  long long dp_cursor, dp_end;  // hybrid: the whole tiles after the stream-K part
+  // width: the stream-K width, p.sk_width unless the kernel derived it from
+  // a tile count it computed itself; sk_tiles: the hybrid's stream-K tiles
+  __device__ __forceinline__ WorkIter(const KParams& p, long long num_tiles, long long width = 0,
+                                      long long sk_tiles = 0) {
+    sk_width = width > 0 ? width : p.sk_width;
+    dp_cursor = 0;
+    dp_end = 0;
+    if (p.work_mode == 2 || p.work_mode == 3) {
+      const long long total = (p.work_mode == 3 ? sk_tiles : num_tiles) * p.num_kb;
+      cursor = static_cast<long long>(blockIdx.x) * sk_width;
+      end = min(total, cursor + sk_width);
       step = 0;
+      if (p.work_mode == 3) {
+        dp_cursor = sk_tiles + blockIdx.x;
+        dp_end = num_tiles;
+      }
     } else {
       const long long units = p.work_mode == 1 ? num_tiles * p.splits : num_tiles;
       cursor = blockIdx.x;
@@ -142,14 +164,23 @@ struct WorkIter {
     }
   }
   __device__ __forceinline__ bool next(const KParams& p, Work& w) {
-    if (cursor >= end) return false;
-    if (p.work_mode == 2) {
+    if (cursor >= end) {
+      if (p.work_mode != 3 || dp_cursor >= dp_end) return false;
+      w.t = dp_cursor;
+      w.idx = 0;
+      w.count = 1;
+      w.kb0 = 0;
+      w.kb1 = p.num_kb;
+      dp_cursor += gridDim.x;
+      return true;
+    }
+    if (p.work_mode >= 2) {
       const long long nkb = p.num_kb;
       w.t = cursor / nkb;
       w.kb0 = static_cast<int>(cursor - w.t * nkb);
       w.kb1 = static_cast<int>(min(nkb, static_cast<long long>(w.kb0) + (end - cursor)));
-      const long long first = (w.t * nkb) / p.sk_width;
-      const long long last = ((w.t + 1) * nkb - 1) / p.sk_width;
+      const long long first = (w.t * nkb) / sk_width;
+      const long long last = ((w.t + 1) * nkb - 1) / sk_width;
       w.idx = static_cast<int>(blockIdx.x - first);
       w.count = static_cast<int>(last - first + 1);
       cursor += w.kb1 - w.kb0;
@@ -171,6 +202,19 @@ struct WorkIter {
     return true;
   }
 };
+
+// The hybrid split of work_mode 3 for `num_tiles` tiles on this grid: the
+// tiles past whole waves, plus one whole wave when there are two or more,
+// go to stream-K (*sk_tiles, over which each block takes *sk_width
+// iterations); the rest run as whole tiles.  Every role computes the same.
+__device__ __forceinline__ void hybrid_split(long long num_tiles, int num_kb, long long* sk_tiles,
+                                             long long* sk_width) {
+  const long long g = gridDim.x;
+  const long long waves = num_tiles / g;
+  const long long dp = (num_tiles % g == 0) ? num_tiles : (waves >= 2 ? (waves - 1) * g : 0);
+  *sk_tiles = num_tiles - dp;
+  *sk_width = max(1ll, (*sk_tiles * num_kb + g - 1) / g);
+}
 
 struct SharedCtl {
   int abort;
@@ -306,6 +350,18 @@ __device__ __forceinline__ TileCoord tile_coord(long long t, const KParams& p, i
   return c;
 }
 
+
+// Scratch slot (in partial tiles) of piece s of split tile t, whose piece 0
+// is processed by block first_block:
+//   split-K: slot t * slot_stride + s;
+//   stream-K: two slots per block, one for the tile its range starts inside
+//   (a piece s > 0) and one for the tile its range ends inside (piece 0), so
+//   the scratch is 2 x grid partial tiles whatever the tile count.
+__device__ __forceinline__ long long piece_slot(const KParams& p, long long t, int s,
+                                                long long first_block) {
+  if (p.work_mode >= 2) return 2 * (first_block + s) + (s > 0 ? 0 : 1);
+  return t * p.slot_stride + s;
+}
 
 // Partial tiles are laid out [BN/4][128 rows][4 floats] so that the 32
 // lanes of a warp, which hold 32 consecutive rows, touch 512 contiguous
@@ -508,15 +564,16 @@ struct TmemSrc {
 // A partial-tile sum as a source (the last piece of a split tile).
 // The sum of a split tile's pieces, for the piece that finishes it: piece
 // `own` is this block's accumulator in tensor memory (`acc`), every other
-// piece s is the fp32 partial tile at tile0 + s * stride.  Columns cc ..
+// piece s is the fp32 partial tile in scratch slot piece_slot(t, s).  Columns cc ..
 // cc+W-1 of this thread's row are summed in piece order, so the result does
 // not depend on which piece finished last; all W/4 loads of one partial are
 // issued before any is used (one memory round trip per piece, not W/4).
 // Returned as raw fp32 bits.
 struct PieceSumSrc {
   TmemSrc acc;
-  const float* tile0;
-  long long stride;
+  const KParams* p;
+  long long t, first_block;  // the tile, and the block of its piece 0
+  long long part;            // floats per partial tile
   int count, own, row;
   template <int W>
   __device__ __forceinline__ void get(int cc, uint32_t (&v)[W]) const {
@@ -532,7 +589,8 @@ struct PieceSumSrc {
         for (int j = 0; j < W; ++j) f[j] += __uint_as_float(t[j]);
         continue;
       }
-      const float4* q = reinterpret_cast<const float4*>(tile0 + s * stride);
+      const float4* q =
+          reinterpret_cast<const float4*>(p->ws + piece_slot(*p, t, s, first_block) * part);
       float4 t[W / 4];
 #pragma unroll
       for (int j = 0; j < W / 4; ++j)

@@ -138,8 +138,8 @@ def _grouped_calls(dg, torch, names, E, R, N, K, dtype):
                                 dg.GEMM_EPI_RELU, code, stream)
     calls, skipped = {}, {}
     for cid, name in enumerate(names):
-        if name.startswith(("swap", "pair")) or "_k" in name or name.endswith("_sk"):
-            skipped[cid] = "not a grouped kernel (or split-K / stream-K, which grouped ignores)"
+        if name.startswith(("swap", "pair", "csk")) or "_k" in name:
+            skipped[cid] = "not a grouped kernel (or split-K, which grouped ignores)"
         else:
             calls[cid] = call
     return calls, skipped, keep

@@ -49,15 +49,20 @@ def test_config_sampled(name):
     _dense_case(workloads.get(name), sampled=True)
 
 
-def test_moe_grouped_sampled():
+@pytest.mark.parametrize("config", [-1, 24, 34])
+def test_moe_grouped_sampled(config):
     w = workloads.get("moe32_m8192n1408k4096_bf16_relu")
     X, W, rows_per, bias = workloads.make_grouped_inputs(w)
     total = int(rows_per.sum())
     dX, dW = X.cuda(), W.cuda()
     drows = torch.from_numpy(rows_per).cuda()
     g = Guarded(total, w.N, w.N, torch.bfloat16)
-    rc = dg.grouped_gemm(w.experts, drows, total, w.N, w.K, dX, w.K, dW, w.N, w.K * w.N, g.ptr,
-                         w.N, None, dg.GEMM_EPI_RELU, dg.GEMM_BF16)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        rc = dg.grouped_gemm(w.experts, drows, total, w.N, w.K, dX, w.K, dW, w.N, w.K * w.N,
+                             g.ptr, w.N, None, dg.GEMM_EPI_RELU, dg.GEMM_BF16)
+    finally:
+        dg.gemm_force_config(-1)
     assert rc == 0, dg.gemm_status_string(rc)
     torch.cuda.synchronize()
     assert dg.gemm_device_status() == 0
@@ -74,7 +79,7 @@ def test_moe_grouped_sampled():
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("b_col", [False, True])
 @pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 12, 13, 23, 24, 28, 29, 30, 31,
-                                    32])
+                                    32, 34, 35])
 def test_exact_integers(dtype, b_col, config):
     """Integer inputs in [-2, 2] with K <= 4096: every partial sum is an
     exact integer below 2^24, so the fp32 accumulator is exact in any order
@@ -145,7 +150,7 @@ def test_empty_m_or_n_is_a_noop():
     assert bool((g.ibuf.cpu() == g.sent).all())
 
 
-DENSE_CONFIGS = list(range(25)) + list(range(28, 34))  # 25..27 are grouped-only
+DENSE_CONFIGS = list(range(25)) + list(range(28, 36))  # 25..27 are grouped-only
 
 
 @pytest.mark.parametrize("config", DENSE_CONFIGS)
@@ -357,17 +362,16 @@ def test_runs_on_a_side_stream():
 # --------------------------------------------------------------- grouped
 
 # 128 x 256 / 128 x 128 row tiles; swapped operands (one CTA, then CTA pairs)
-GROUPED_CONFIGS = [0, 1, 25, 26, 27]
+# 23, 24: stream-K over the groups' tiles; 34, 35: the hybrid
+GROUPED_CONFIGS = [0, 1, 23, 24, 25, 26, 27, 34, 35]
 
 
 @pytest.mark.parametrize("b_col", [False, True])
 @pytest.mark.parametrize("out_f32", [False, True])
 @pytest.mark.parametrize("config", GROUPED_CONFIGS)
 def test_grouped_every_element(b_col, out_f32, config):
-    if config >= 25:
+    if 25 <= config <= 27:
         assert dg.gemm_config_name(config).startswith("gswap")
-    if config >= 26:
-        assert dg.gemm_config_name(config).startswith("gswap2")
     rows_per = np.array([0, 3, 130, 1, 0, 257, 64, 0], dtype=np.int32)
     G, N, K = len(rows_per), 200, 136
     total = int(rows_per.sum())
@@ -396,7 +400,7 @@ def test_grouped_every_element(b_col, out_f32, config):
     g.check_canaries()
 
 
-@pytest.mark.parametrize("config", [-1, 25, 26])
+@pytest.mark.parametrize("config", [-1, 24, 25, 26])
 def test_grouped_counts_beyond_total_are_clipped_and_reported(config):
     rows_per = np.array([5, 300, 40], dtype=np.int32)  # sums to 345
     total, N, K = 200, 64, 64                           # caller says 200
