@@ -87,6 +87,8 @@ def lib() -> ctypes.CDLL:
             L.gemm_splitk_noalloc.restype = I
             L.gemm_set_trace.argtypes = [P, L64]
             L.gemm_set_trace.restype = I
+            L.gemm_free_scratch.argtypes = [P, I]
+            L.gemm_free_scratch.restype = I
             _lib = L
     return _lib
 
@@ -161,6 +163,13 @@ def gemm_version() -> str:
 
 def gemm_device_status(stream=None, clear: bool = True) -> int:
     return lib().gemm_device_status(_stream(stream), int(clear))
+
+
+def gemm_free_scratch(stream=None, all_streams: bool = False) -> int:
+    """C-ABI ``gemm_free_scratch``: free the library's scratch for ``stream``
+    (the current stream by default), or for every stream with all_streams."""
+    return lib().gemm_free_scratch(None if all_streams else _stream(stream),
+                                   1 if all_streams else 0)
 
 
 def gemm_set_trace(buffer, nbytes: int) -> int:

@@ -964,6 +964,30 @@ int gemm_device_status(void* stream_, int clear) {
   return GEMM_ERR_DEVICE_TIMEOUT;
 }
 
+int gemm_free_scratch(void* stream_, int all_streams) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  std::lock_guard<std::mutex> lk(g_ws_mu);
+  int rc = GEMM_OK;
+  for (auto it = g_ws.begin(); it != g_ws.end();) {
+    if (it->device != dev || (!all_streams && it->stream != stream)) {
+      ++it;
+      continue;
+    }
+    e = cudaStreamSynchronize(it->stream);
+    if (e != cudaSuccess) {
+      rc = cuda_fail(e);
+      ++it;
+      continue;
+    }
+    cudaFree(it->ptr);
+    it = g_ws.erase(it);
+  }
+  return rc;
+}
+
 int gemm_set_trace(void* buffer, int64_t bytes) {
   if (buffer && (reinterpret_cast<uintptr_t>(buffer) & 7u) != 0) return GEMM_ERR_MISALIGNED;
   const int64_t blocks = buffer ? bytes / static_cast<int64_t>(8 * kTraceEvents) : 0;

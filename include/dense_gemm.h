@@ -26,10 +26,13 @@
  *           pointer owned by the caller.  The library never frees or keeps
  *           a reference to a caller buffer after the call.  Its own device
  *           memory is a status word per device and, only for calls that need
- *           it, per-stream scratch: split-K / stream-K partial tiles and the
- *           im2col matrix of conv2d_im2col, each allocated with cudaMalloc on
- *           the first such call on a stream and grown on demand
- *           (gemm_splitk_noalloc never allocates).
+ *           it, per-stream scratch: split-K / stream-K partial tiles, tile
+ *           counters and the im2col matrix of conv2d_im2col, each allocated
+ *           with cudaMalloc on the first such call on a stream and grown on
+ *           demand (gemm_splitk_noalloc never allocates).  The scratch is
+ *           keyed by the stream handle and kept until gemm_free_scratch().
+ *           Destroy a stream only after gemm_free_scratch(stream), or a new
+ *           stream that is given the same handle would share its scratch.
  * Alignment. A, B and C must be 16-byte aligned; lda*sizeof(input),
  *           ldb*sizeof(input) and ldc*sizeof(output) must be multiples of 16
  *           bytes (the tensor-memory-access unit copies 16-byte granules):
@@ -227,6 +230,16 @@ GEMM_API uint64_t gemm_set_timeout_ns(uint64_t ns);
  * GEMM_ERR_DEVICE_TIMEOUT).  No fault, trap or hang is involved.
  */
 GEMM_API int gemm_watchdog_selftest(uint64_t timeout_ns, void* stream);
+
+/*
+ * gemm_free_scratch -- synchronise `stream` and free the scratch the library
+ * holds for it on the current device (NULL is the default stream).  With
+ * all_streams != 0, `stream` is ignored and every stream's scratch on the
+ * current device is freed, each after synchronising its stream.  Later calls
+ * allocate anew.  Returns GEMM_OK (also when there was nothing to free) or
+ * GEMM_ERR_CUDA.
+ */
+GEMM_API int gemm_free_scratch(void* stream, int all_streams);
 
 /* ---- tracing ----------------------------------------------------------- */
 

@@ -347,6 +347,28 @@ def test_pair_split_k_rejects_what_it_cannot_split(config):
     assert int(C.abs().sum()) == 0
 
 
+def test_freeing_scratch_keeps_later_calls_right():
+    # split-K scratch for a side stream, freed, then allocated anew by the
+    # next call; freeing every stream's scratch leaves the library usable
+    M, N, K = 256, 384, 4096
+    gen = torch.Generator().manual_seed(8)
+    A = torch.randn(M, K, generator=gen).half()
+    B = torch.randn(N, K, generator=gen).half()
+    ref = oracle.gemm(M, N, K, A, K, B, K, b_colmajor=True, dtype="f16", threads=THREADS)
+    s = torch.cuda.Stream()
+    sk = [i for i in range(dg.gemm_num_configs()) if dg.gemm_config_name(i) == "tc1_128x128_s6_g8_k4"][0]
+    assert dg.gemm_force_config(sk) == 0
+    try:
+        for free_all in (False, True, False):
+            with torch.cuda.stream(s):
+                g = run_gemm(A.cuda(), B.cuda(), None, M, N, K, b_col=True, stream=s)
+                compare(g.matrix().double().cpu().numpy(), ref, 2, f"after free (all={free_all})")
+            assert dg.gemm_free_scratch(s, all_streams=free_all) == 0
+    finally:
+        dg.gemm_force_config(-1)
+    assert dg.gemm_free_scratch(s) == 0  # nothing left to free
+
+
 def test_runs_on_a_side_stream():
     s = torch.cuda.Stream()
     w = workloads.get("square256_f16")
