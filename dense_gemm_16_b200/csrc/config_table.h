@@ -74,9 +74,9 @@ static const Rule kRules[] = {
     {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 31},  // m1000n1000k2000_bcol: csk_2x128x128_s4 217 TFLOP/s
     {4096, 4096, 4096, 4096, 512, 512, 1, 0, 0},  // m4096n4096k512_bcol: tc1_128x256_s4_g8 598 TFLOP/s
     {16, 16, 8192, 8192, 8192, 8192, 1, 0, 21},  // m16n8192k8192_bcol: swap_128x16_s8_sk 62 TFLOP/s
-    {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 678 TFLOP/s
-    {16384, 16384, 4096, 4096, 4096, 4096, 0, 1, 0},  // moe8_n4096_k4096: tc1_128x256_s4_g8 1181 TFLOP/s
-    {8192, 8192, 768, 768, 2048, 2048, 0, 1, 35},  // moe64_n768_k2048: tc1_128x128_s6_g8_hy 349 TFLOP/s
+    {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 688 TFLOP/s
+    {16384, 16384, 4096, 4096, 4096, 4096, 0, 1, 11},  // moe8_n4096_k4096: pair_256x256_s6_g16 1237 TFLOP/s
+    {8192, 8192, 768, 768, 2048, 2048, 0, 1, 11},  // moe64_n768_k2048: pair_256x256_s6_g16 399 TFLOP/s
     {0, 0, 0, 0, 0, 0, -1, -1, -1},  // sentinel
 };
 // END RULES

@@ -44,6 +44,7 @@ KernelEntry kernels_bn128(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_bn64(bool q_mn, bool bf16, bool out_f32, bool grouped);
 KernelEntry kernels_swap(int bn, bool bf16, bool out_f32);
 KernelEntry kernels_pair(int bn, int stages, bool q_mn, bool bf16, bool out_f32);
+KernelEntry kernels_pair_grouped(int bn, bool q_mn, bool bf16, bool out_f32);
 KernelEntry kernels_tf32(int bn, bool q_mn);
 KernelEntry kernels_gswap(int tok, bool p_mn, bool bf16, bool out_f32);
 KernelEntry kernels_gswap2(int tok, bool p_mn, bool bf16, bool out_f32);

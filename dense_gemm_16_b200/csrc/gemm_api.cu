@@ -330,7 +330,7 @@ KernelEntry kernel_for(const Config& c, bool q_mn, bool bf16, bool f32, bool gro
                                       : kernels_gswap2(c.bn, q_mn, bf16, f32);
   }
   if (c.kind == kKindPair) {
-    if (grouped) return {nullptr, 0};
+    if (grouped) return kernels_pair_grouped(c.bn, q_mn, bf16, f32);
     return kernels_pair(c.bn, c.stages, q_mn, bf16, f32);
   }
   if (c.bn == 256) return kernels_bn256(q_mn, bf16, f32, grouped);
@@ -881,10 +881,18 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
                                ldb, stride_b, C, ldc, bias, epilogue, bf16, stream);
 
   CUtensorMap tp, tq;
+  const bool pair = cfg.kind == kKindPair;
   const uint64_t lda_b = static_cast<uint64_t>(lda) * 2;
-  const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(total_rows)};
-  const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
-  rc = make_map(&tp, A, bf16, 2, dA, &lda_b, bA);
+  if (pair) {  // the pair kernel copies A with 3-D boxes (one batch)
+    const uint64_t dA[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(total_rows), 1};
+    const uint64_t sA[2] = {lda_b, lda_b * static_cast<uint64_t>(total_rows)};
+    const uint32_t bA[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM), 1u};
+    rc = make_map(&tp, A, bf16, 3, dA, sA, bA);
+  } else {
+    const uint64_t dA[2] = {static_cast<uint64_t>(K), static_cast<uint64_t>(total_rows)};
+    const uint32_t bA[2] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(kBM)};
+    rc = make_map(&tp, A, bf16, 2, dA, &lda_b, bA);
+  }
   if (rc) return rc;
   const uint64_t sB[2] = {static_cast<uint64_t>(ldb) * 2, static_cast<uint64_t>(stride_b) * 2};
   // a single group may pass stride_b = 0; give the map a valid stride
@@ -892,7 +900,10 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
   if (bcol) {
     const uint64_t dB[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(N),
                             static_cast<uint64_t>(num_groups)};
-    const uint32_t bB[3] = {static_cast<uint32_t>(kBK), static_cast<uint32_t>(cfg.bn), 1u};
+    // each CTA of a pair loads half of every N=256 MMA's B rows
+    const uint32_t rows_b = pair ? static_cast<uint32_t>(std::min(cfg.bn, 256) / 2)
+                                 : static_cast<uint32_t>(cfg.bn);
+    const uint32_t bB[3] = {static_cast<uint32_t>(kBK), rows_b, 1u};
     rc = make_map(&tq, B, bf16, 3, dB, sB_fix, bB);
   } else {
     const uint64_t dB[3] = {static_cast<uint64_t>(N), static_cast<uint64_t>(K),
@@ -928,6 +939,13 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
   const long long max_tiles = (static_cast<long long>(total_rows) / kBM + num_groups) * nq;
   CUtensorMap tc;
   std::memset(&tc, 0, sizeof(tc));  // grouped tiles store from registers
+  if (pair) {
+    // 256-row pair tiles; one cluster of two CTAs per pair
+    const long long max_pair_tiles =
+        (static_cast<long long>(total_rows) / (2 * kBM) + num_groups) * nq;
+    const int pairs = static_cast<int>(std::min<long long>(max_pair_tiles, ds->num_sms / 2));
+    return launch(k, 2 * pairs, stream, tp, tq, tc, kp, 2);
+  }
   const int grid = static_cast<int>(std::min<long long>(max_tiles, ds->num_sms));
   if (cfg.splits < 0 && kp.num_kb >= 2 && max_tiles <= static_cast<long long>(kCounterSlots)) {
     // stream-K (-1) or the hybrid (-2) over the (tile, K block) space; the

@@ -31,7 +31,12 @@ namespace dg16 {
 // STAGES  ring depth
 // Q_MN    B is row-major (MN-major operand)
 // IN_BF16 / OutT as in the single-CTA kernel
-template <int BN, int NSUB, int STAGES, bool Q_MN, bool IN_BF16, typename OutT>
+// GROUPED grouped GEMM: pair tiles of 256 rows within one group (rows of A
+//         sorted by group, B a [group][K][N] or [group][N][K] stack); the
+//         tile prefix is built in shared memory from the device-side group
+//         sizes, and stores are masked at the group's last row
+template <int BN, int NSUB, int STAGES, bool Q_MN, bool IN_BF16, typename OutT,
+          bool GROUPED = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmQ,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ KParams p) {
@@ -47,6 +52,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t Q_BYTES = NSUB * QSUB_BYTES;
   constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
   constexpr uint32_t TMEM_COLS = (ACC_BUFS * TILE_N <= 256) ? 256 : 512;
+  // grouped tiles must not write past their group's last row: they store
+  // from registers and need no staging buffer
+  constexpr uint32_t STAGE_EPI = GROUPED ? 0u : kEpiStageBytes;
   constexpr uint32_t IDESC = f16_idesc(2 * kBM, BN, IN_BF16 ? 1u : 0u, 0u, Q_MN ? 1u : 0u);
 
   extern __shared__ uint8_t smem_raw[];
@@ -55,13 +63,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sP = smem;
   uint8_t* sQ = smem + STAGES * P_BYTES;
   uint8_t* sStage = sQ + STAGES * Q_BYTES;  // 1024-aligned epilogue staging
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + kEpiStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + STAGE_EPI);
   uint64_t* full_bar = bars;
   uint64_t* empty_bar = bars + STAGES;
   uint64_t* accf_bar = bars + 2 * STAGES;
   uint64_t* acce_bar = bars + 2 * STAGES + 2;
   uint64_t* drain_bar = bars + 2 * STAGES + 4;
   SharedCtl* ctl = reinterpret_cast<SharedCtl*>(bars + 2 * STAGES + 5);
+  GroupTable* gt = reinterpret_cast<GroupTable*>(ctl + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -90,19 +99,80 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmP);
     tma_prefetch_desc(&tmQ);
-    tma_prefetch_desc(&tmC);
+    if constexpr (!GROUPED) tma_prefetch_desc(&tmC);
   }
   if (warp == 1) {
     tmem_alloc<2>(smem_u32(&ctl->tmem_base), TMEM_COLS);
     tmem_relinquish<2>();
+  }
+  const int num_q_tiles = (p.N + TILE_N - 1) / TILE_N;
+  if constexpr (GROUPED) {
+    if (warp == 2 && lane == 0) {
+      // per-group tile prefix (256-row blocks) from the device counts; each
+      // CTA of the pair builds the same table
+      int tiles = 0, rows = 0;
+      bool bad = false;
+      for (int g = 0; g < p.num_groups; ++g) {
+        int m = __ldg(&p.group_rows[g]);
+        if (m < 0) {
+          m = 0;
+          bad = true;
+        }
+        gt->tile_start[g] = tiles;
+        gt->row_start[g] = rows;
+        const int usable = max(0, min(m, p.M - rows));  // rows past the total are never touched
+        if (usable < m) bad = true;
+        tiles += (usable + 2 * kBM - 1) / (2 * kBM) * num_q_tiles;
+        rows += usable;
+      }
+      gt->tile_start[p.num_groups] = tiles;
+      gt->row_start[p.num_groups] = rows;
+      if (bad && blockIdx.x == 0) atomicCAS(p.status, 0u, kStatusBadGroups);
+    }
   }
   tc_fence_before();
   __syncthreads();
   cluster_sync();  // both CTAs' barriers are initialised before any remote use
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
-  const long long num_tiles = p.num_tiles;
+  const long long num_tiles = GROUPED ? gt->tile_start[p.num_groups] : p.num_tiles;
   if (threadIdx.x == 0) trace_mark(p, kTrSetup);
+
+  // Where pair tile t lives: its first row (of the batch, or global for
+  // grouped), its column block, the TMA batch/group coordinates, the batch
+  // or group index and the end of the rows it may store.  Tile ids reach
+  // each role in increasing order, so the group cursor only walks forward.
+  struct PairTile {
+    int p0, qb, zp, zq, b, row_end;
+  };
+  auto pair_tile = [&](long long t, int& gcur) {
+    PairTile c;
+    if constexpr (GROUPED) {
+      while (gcur < p.num_groups - 1 && t >= gt->tile_start[gcur + 1]) ++gcur;
+      const int g = gcur;
+      const int local = static_cast<int>(t - gt->tile_start[g]);
+      const int rows = gt->row_start[g + 1] - gt->row_start[g];
+      int mb, nb;
+      raster_tile(local, (rows + 2 * kBM - 1) / (2 * kBM), num_q_tiles, p.group_m, mb, nb);
+      c.p0 = gt->row_start[g] + mb * 2 * kBM;
+      c.qb = nb;
+      c.zp = 0;
+      c.zq = g;
+      c.b = g;
+      c.row_end = min(gt->row_start[g + 1], p.M);
+    } else {
+      const long long b = t / p.tiles_per_batch;
+      int pb, qb;
+      raster_tile(t - b * p.tiles_per_batch, p.num_p, p.num_q, p.group_m, pb, qb);
+      c.p0 = pb * (2 * kBM);
+      c.qb = qb;
+      c.zp = static_cast<int>(b) * p.z_p;
+      c.zq = static_cast<int>(b) * p.z_q;
+      c.b = static_cast<int>(b);
+      c.row_end = p.M;
+    }
+    return c;
+  };
 
   if (warp == 0) {
     // ---------------------------------------------- TMA producer (both CTAs)
@@ -111,15 +181,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t pol_q = make_policy(p.pol_q);
       uint32_t it = 0;
       bool ok = true;
+      int gcur = 0;
       for (long long t = pair_id; t < num_tiles && ok; t += num_pairs) {
-        const long long b = t / p.tiles_per_batch;
-        int pb, qb;
-        raster_tile(t - b * p.tiles_per_batch, p.num_p, p.num_q, p.group_m, pb, qb);
-        const int zp = static_cast<int>(b) * p.z_p, zq = static_cast<int>(b) * p.z_q;
-        const int prow0 = pb * (2 * kBM) + static_cast<int>(rank) * kBM;
+        const PairTile c = pair_tile(t, gcur);
+        const int zp = c.zp, zq = c.zq;
+        const int prow0 = c.p0 + static_cast<int>(rank) * kBM;
         // MMA j of the K step covers tile columns [j*BN, (j+1)*BN); this CTA
         // supplies the rank-th half of each
-        const int qcol0 = qb * TILE_N + static_cast<int>(rank) * HALF_N;
+        const int qcol0 = c.qb * TILE_N + static_cast<int>(rank) * HALF_N;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
@@ -219,31 +288,34 @@ __global__ void __launch_bounds__(kThreads, 1)
     const InT* bias = (p.epi & 1) ? reinterpret_cast<const InT*>(p.bias) : nullptr;
     const bool relu = (p.epi & 2) != 0;
     const uint32_t acce_leader0 = map_shared_rank(smem_u32(&acce_bar[0]), 0);
+    int gcur = 0;
     for (long long t = pair_id; t < num_tiles; t += num_pairs, ++local) {
-      const long long b = t / p.tiles_per_batch;
-      int pb, qb;
-      raster_tile(t - b * p.tiles_per_batch, p.num_p, p.num_q, p.group_m, pb, qb);
-      const InT* const bias_t = bias ? bias + b * p.stride_bias : nullptr;
+      const PairTile c = pair_tile(t, gcur);
+      const long long b = c.b;
+      const int qb = c.qb;
+      const InT* const bias_t =
+          bias ? bias + b * (GROUPED ? static_cast<long long>(p.N) : p.stride_bias) : nullptr;
       const uint32_t a = ACC_BUFS == 2 ? (local & 1u) : 0u;
       const uint32_t aph = ACC_BUFS == 2 ? ((local >> 1) & 1u) : (local & 1u);
       const bool ok = wait_phase<true>(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
       if (!__all_sync(0xffffffffu, ok)) break;
       if (warp == 2 && lane == 0 && local == 0) trace_mark(p, kTrFirstEpi);
       tc_fence_after();
-      const int row0 = pb * (2 * kBM) + static_cast<int>(rank) * kBM + quad * 32;
+      const int row0 = c.p0 + static_cast<int>(rank) * kBM + quad * 32;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * TILE_N;
       const TmemSrc tsrc{taddr};
-      if (p.tma_store)
+      if (!GROUPED && p.tma_store)
         store_tma_from<TILE_N, InT, OutT>(tsrc, row0, qb * TILE_N, static_cast<int>(b), p, bias_t,
                                           relu, stage, stores, &tmC);
       else
-        store_rows_from<TILE_N, InT, OutT>(tsrc, row0 + lane, p.M, qb * TILE_N, p, bias_t, relu,
-                                           reinterpret_cast<OutT*>(p.C) + b * p.stride_c);
+        store_rows_from<TILE_N, InT, OutT>(
+            tsrc, row0 + lane, c.row_end, qb * TILE_N, p, bias_t, relu,
+            reinterpret_cast<OutT*>(p.C) + (GROUPED ? 0 : b * p.stride_c));
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acce_leader0 + a * 8u);
     }
-    if (lane == 0) tma_store_wait_read<0>();  // staging read; writes finish with the grid
+    if (!GROUPED && lane == 0) tma_store_wait_read<0>();  // staging read; writes finish with the grid
     if (warp == 2 && lane == 0) trace_mark(p, kTrEpiDone);
   }
 
@@ -258,10 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) trace_mark(p, kTrExit);
 }
 
-template <int BN, int NSUB, int STAGES>
+template <int BN, int NSUB, int STAGES, bool GROUPED = false>
 constexpr int gemm_pair_smem_bytes() {
   return 1024 + STAGES * (kBM * kBK * 2 + NSUB * (BN / 2) * kBK * 2) +
-         static_cast<int>(kEpiStageBytes) + (2 * STAGES + 5) * 8 + static_cast<int>(sizeof(SharedCtl));
+         (GROUPED ? 0 : static_cast<int>(kEpiStageBytes)) + (2 * STAGES + 5) * 8 +
+         static_cast<int>(sizeof(SharedCtl)) + (GROUPED ? static_cast<int>(sizeof(GroupTable)) : 0);
 }
 
 }  // namespace dg16

@@ -138,7 +138,7 @@ def _grouped_calls(dg, torch, names, E, R, N, K, dtype):
                                 dg.GEMM_EPI_RELU, code, stream)
     calls, skipped = {}, {}
     for cid, name in enumerate(names):
-        if name.startswith(("swap", "pair", "csk")) or "_k" in name:
+        if name.startswith(("swap", "csk", "pair_256x128")) or "_k" in name:
             skipped[cid] = "not a grouped kernel (or split-K, which grouped ignores)"
         else:
             calls[cid] = call

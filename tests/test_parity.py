@@ -49,7 +49,7 @@ def test_config_sampled(name):
     _dense_case(workloads.get(name), sampled=True)
 
 
-@pytest.mark.parametrize("config", [-1, 24, 34])
+@pytest.mark.parametrize("config", [-1, 13, 24, 34])
 def test_moe_grouped_sampled(config):
     w = workloads.get("moe32_m8192n1408k4096_bf16_relu")
     X, W, rows_per, bias = workloads.make_grouped_inputs(w)
@@ -193,14 +193,14 @@ def test_swap_config_rejects_row_major_b():
 
 
 def test_configs_of_the_other_kind_are_rejected():
-    # a grouped-only config on a dense call, a CTA-pair dense config on a
+    # a grouped-only config on a dense call, a swapped (skinny) config on a
     # grouped call: UNSUPPORTED, and nothing is written
     A = torch.ones(64, 64, dtype=torch.half, device="cuda")
     B = torch.ones(64, 64, dtype=torch.half, device="cuda")
     C = torch.zeros(64, 64, dtype=torch.half, device="cuda")
     rows = torch.tensor([32, 32], dtype=torch.int32, device="cuda")
     Bg = torch.ones(2, 64, 64, dtype=torch.half, device="cuda")
-    pair = [i for i in range(dg.gemm_num_configs()) if dg.gemm_config_name(i).startswith("pair")][0]
+    pair = [i for i in range(dg.gemm_num_configs()) if dg.gemm_config_name(i).startswith("swap")][0]
     try:
         assert dg.gemm_force_config(25) == 0
         assert dg.gemm(64, 64, 64, A, 64, B, 64, C, 64, None, 0,
@@ -384,8 +384,8 @@ def test_runs_on_a_side_stream():
 # --------------------------------------------------------------- grouped
 
 # 128 x 256 / 128 x 128 row tiles; swapped operands (one CTA, then CTA pairs)
-# 23, 24: stream-K over the groups' tiles; 34, 35: the hybrid
-GROUPED_CONFIGS = [0, 1, 23, 24, 25, 26, 27, 34, 35]
+# 23, 24: stream-K over the groups' tiles; 34, 35: the hybrid; 4, 13: CTA pairs
+GROUPED_CONFIGS = [0, 1, 4, 13, 23, 24, 25, 26, 27, 34, 35]
 
 
 @pytest.mark.parametrize("b_col", [False, True])
@@ -422,7 +422,7 @@ def test_grouped_every_element(b_col, out_f32, config):
     g.check_canaries()
 
 
-@pytest.mark.parametrize("config", [-1, 24, 25, 26])
+@pytest.mark.parametrize("config", [-1, 4, 13, 24, 25, 26])
 def test_grouped_counts_beyond_total_are_clipped_and_reported(config):
     rows_per = np.array([5, 300, 40], dtype=np.int32)  # sums to 345
     total, N, K = 200, 64, 64                           # caller says 200
@@ -455,7 +455,7 @@ def _grouped_problem(rows_per, N, K, seed, dtype=torch.bfloat16, b_col=False):
     return X, W, bias
 
 
-@pytest.mark.parametrize("config", [25, 26])
+@pytest.mark.parametrize("config", [25, 26, 4, 13])
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 def test_grouped_swap_many_groups_every_element(config, dtype):
     # 40 groups: empty, 1..15 rows (one 16-row box), exact multiples of 16,
