@@ -111,6 +111,12 @@ WORKLOADS = {w.name: w for w in [
     _w(name="square6144_bf16", M=6144, N=6144, K=6144, dtype="bf16", dist="normal", seed=12),
     _w(name="moe32_m8192n1408k4096_bf16_relu", M=8192, N=1408, K=4096, dtype="bf16",
        dist="normal", seed=11, relu=True, experts=32, w_std=0.02),
+    # two more routings with the same generator: few large experts, and many
+    # experts with a narrow N (the swept grouped classes)
+    _w(name="moe8_m16384n4096k4096_bf16_relu", M=16384, N=4096, K=4096, dtype="bf16",
+       dist="normal", seed=11, relu=True, experts=8, w_std=0.02),
+    _w(name="moe64_m8192n768k2048_bf16_relu", M=8192, N=768, K=2048, dtype="bf16",
+       dist="normal", seed=11, relu=True, experts=64, w_std=0.02),
 ]}
 
 
