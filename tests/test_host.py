@@ -105,6 +105,22 @@ def test_select_config_shape_classes():
     assert dg.gemm_select_config(1, 1, 1, 9, 0) == dg.GEMM_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("M,N,K,dtype,epi,prefix", [
+    (8192, 8192, 8192, "bf16", 0, "pair_256x512"),  # measured rule: CTA-pair 256 x 512 tiles
+    (4096, 4096, 4096, "bf16", 0, "pair_256x512"),
+    (1024, 1024, 2048, "f16", 0, "csk_"),           # the pages' shape: CTA-pair split-K
+    (512, 512, 2048, "f16", 0, "csk_"),             # no rule: few tiles, long K -> pair split-K
+    (512, 512, 256, "f16", 0, "tc1_128x128"),       # few tiles, short K -> 128 x 128 tiles
+    (3000, 3000, 3000, "bf16", 0, "pair_256x256"),  # no rule: >= 128 pair tiles, K >= 1024
+    (16, 8192, 8192, "f16", 0x100, "swap_128x16"),  # skinny, B column-major -> swapped operands
+    (24, 4096, 4096, "f16", 0x100, "swap_128x32"),
+])
+def test_table_and_fallback_choices(M, N, K, dtype, epi, prefix):
+    code = dg.GEMM_BF16 if dtype == "bf16" else dg.GEMM_F16
+    cid = dg.gemm_select_config(M, N, K, code, epi)
+    assert dg.gemm_config_name(cid).startswith(prefix), dg.gemm_config_name(cid)
+
+
 # Fake, never-dereferenced device addresses: every case below must be
 # rejected by the host checks before any CUDA call.
 P = 1 << 20  # 16-byte aligned
