@@ -52,6 +52,9 @@ static const Config kConfigs[] = {
     {"cskswap_2x128x16_s10", kKindClusterSplitKSwap, 16, 10, 1, 1, 1, 2},
     {"tc1_128x256_s4_g8_hy", kKindSingle, 256, 4, 8, -2, 2, 2},
     {"tc1_128x128_s6_g8_hy", kKindSingle, 128, 6, 8, -2, 2, 2},
+    {"pair_256x512_s4_g16_sk", kKindPair, 512, 4, 16, -1, 2, 2},
+    {"pair_256x512_s4_g16_hy", kKindPair, 512, 4, 16, -2, 2, 2},
+    {"pair_256x256_s6_g16_sk", kKindPair, 256, 6, 16, -1, 2, 2},
 };
 static constexpr int kNumConfigs = static_cast<int>(sizeof(kConfigs) / sizeof(kConfigs[0]));
 

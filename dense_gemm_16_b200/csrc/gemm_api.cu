@@ -569,10 +569,14 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   kp.splits = 1;
   kp.kb_per_split = kp.num_kb;
   kp.slot_stride = 1;
-  int grid_units = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms));
+  // workers: blocks, or CTA pairs for the pair kernel, whose two CTAs keep
+  // their own counters and partial slots for their 128-row halves
+  const int ranks = pair ? 2 : 1;
+  const int workers = ds->num_sms / ranks;
+  int grid_units = static_cast<int>(std::min<long long>(kp.num_tiles, workers));
   const size_t counter_cap = fixed ? fixed->counter_slots : kCounterSlots;
-  if (!pair && !csk && splits != 1 && kp.num_kb >= 2 &&
-      kp.num_tiles <= static_cast<long long>(counter_cap)) {
+  if (!csk && splits != 1 && kp.num_kb >= 2 &&
+      kp.num_tiles * ranks <= static_cast<long long>(counter_cap)) {
     if (splits > 1) {
       // split-K: every tile's K range in `splits` equal pieces
       const int per = (kp.num_kb + splits - 1) / splits;
@@ -580,19 +584,19 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
       kp.kb_per_split = per;
       kp.splits = (kp.num_kb + per - 1) / per;  // no empty K range
       kp.slot_stride = kp.splits;
-      grid_units = static_cast<int>(std::min<long long>(kp.num_tiles * kp.splits, ds->num_sms));
+      grid_units = static_cast<int>(std::min<long long>(kp.num_tiles * kp.splits, workers));
     } else if (splits == -2) {
       // hybrid: stream-K over the last waves' tiles, whole tiles before
       // them; the kernel derives the split from the tile count and grid
       kp.work_mode = 3;
       kp.sk_width = 1;
-      grid_units = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms));
+      grid_units = static_cast<int>(std::min<long long>(kp.num_tiles, workers));
     } else {
       // stream-K: every block gets an equal share of the (tile, K block)
       // iterations, cut at tile edges
       const long long total = kp.num_tiles * kp.num_kb;
       kp.work_mode = 2;
-      kp.sk_width = (total + ds->num_sms - 1) / ds->num_sms;
+      kp.sk_width = (total + workers - 1) / workers;
       grid_units = static_cast<int>((total + kp.sk_width - 1) / kp.sk_width);
       kp.slot_stride = static_cast<int>((kp.num_kb + kp.sk_width - 1) / kp.sk_width) + 1;
     }
@@ -600,16 +604,17 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
   }
   if (kp.work_mode != 0) {
     // split-K: slot_stride slots per tile; stream-K: two per block
-    const size_t slots = kp.work_mode >= 2 ? 2 * static_cast<size_t>(grid_units)
-                                           : static_cast<size_t>(kp.num_tiles) * kp.slot_stride;
+    const size_t slots = (kp.work_mode >= 2 ? 2 * static_cast<size_t>(grid_units)
+                                            : static_cast<size_t>(kp.num_tiles) * kp.slot_stride) *
+                         ranks;
     const size_t partial = slots * kBM * cfg.bn * 4;
     if (fixed) {
       if (partial > fixed->partial_bytes) return GEMM_ERR_UNSUPPORTED;  // beyond the scratch
       kp.ws = fixed->ws;
       kp.counters = fixed->counters;
       // counters left by an earlier call that gave up early must not leak in
-      cudaError_t e = cudaMemsetAsync(kp.counters, 0,
-                                      static_cast<size_t>(kp.num_tiles) * sizeof(unsigned), stream);
+      cudaError_t e = cudaMemsetAsync(
+          kp.counters, 0, static_cast<size_t>(kp.num_tiles) * ranks * sizeof(unsigned), stream);
       if (e != cudaSuccess) return cuda_fail(e);
     } else {
       int dev = 0;
@@ -618,15 +623,12 @@ int run_dense(DeviceState* ds, const DenseProblem& d, const Config& cfg, int spl
       rc = stream_workspace(dev, stream, partial, &kp.ws, &kp.counters);
       if (rc) return rc;
     }
-  } else if (fixed && splits > 1 && kp.num_tiles > static_cast<long long>(counter_cap)) {
+  } else if (fixed && splits > 1 && kp.num_tiles * ranks > static_cast<long long>(counter_cap)) {
     return GEMM_ERR_UNSUPPORTED;  // beyond the scratch's tile counters
   }
   rc = ensure_smem_attr(ds, k);
   if (rc) return rc;
-  if (pair) {
-    const int pairs = static_cast<int>(std::min<long long>(kp.num_tiles, ds->num_sms / 2));
-    return launch(k, 2 * pairs, stream, tp, tq, tc, kp, 2);
-  }
+  if (pair) return launch(k, 2 * grid_units, stream, tp, tq, tc, kp, 2);
   if (csk) {
     // one CTA pair per tile, each CTA one half of the K blocks
     if (kp.num_tiles > ds->num_sms / 2 || kp.num_kb < 2) return GEMM_ERR_UNSUPPORTED;

@@ -293,6 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!c.valid) break;
       const uint32_t a = local & 1u;
       const uint32_t aph = (local >> 1) & 1u;
+      BiasRegs<BN, InT> br;
+      if (!SWAP && TMA_EPI && has_bias)
+        br.load(bias + static_cast<long long>(c.group) * (GROUPED ? p.N : p.stride_bias), c.q0 * BN,
+                p.N);
       // every lane waits; the warp proceeds only if all saw the phase, so the
       // .sync.aligned TMEM loads below are always issued by the whole warp
       const bool ok = wait_phase(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
@@ -375,9 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (w.count > 1)
               store_tma_from<BN, InT, OutT>(psrc, c.p0 + quad * 32, q0, c.group, p, bias_g, relu,
                                             stage, stores, &tmC);
+            else if (bias_g != nullptr)
+              store_tmem_tile<BN, InT, OutT, true>(taddr, c.p0 + quad * 32, q0, c.group, p, br,
+                                                   relu, stage, stores, &tmC);
             else
-              store_tma_from<BN, InT, OutT>(tsrc, c.p0 + quad * 32, q0, c.group, p, bias_g, relu,
-                                            stage, stores, &tmC);
+              store_tmem_tile<BN, InT, OutT, false>(taddr, c.p0 + quad * 32, q0, c.group, p, br,
+                                                    relu, stage, stores, &tmC);
           } else {
             // accumulator row = output row prow, columns q0 .. q0+BN
             if (w.count > 1)

@@ -136,6 +136,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   const long long num_tiles = GROUPED ? gt->tile_start[p.num_groups] : p.num_tiles;
+  // Work split over pairs: whole tiles (mode 0), or stream-K (2) / the
+  // hybrid (3) over (tile, K block) iterations.  A piece of a split tile is
+  // the same K range in both CTAs; each CTA fixes up its own 128 rows with
+  // its own counter (2t + rank) and partial slots.
+  long long sk_width = 0, sk_tiles = 0;
+  if (p.work_mode == 3) hybrid_split(num_tiles, p.num_kb, &sk_tiles, &sk_width, num_pairs);
   if (threadIdx.x == 0) trace_mark(p, kTrSetup);
 
   // Where pair tile t lives: its first row (of the batch, or global for
@@ -182,14 +188,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       int gcur = 0;
-      for (long long t = pair_id; t < num_tiles && ok; t += num_pairs) {
-        const PairTile c = pair_tile(t, gcur);
+      WorkIter wi(p, num_tiles, sk_width, sk_tiles, pair_id, num_pairs);
+      Work w;
+      while (ok && wi.next(p, w)) {
+        const PairTile c = pair_tile(w.t, gcur);
         const int zp = c.zp, zq = c.zq;
         const int prow0 = c.p0 + static_cast<int>(rank) * kBM;
         // MMA j of the K step covers tile columns [j*BN, (j+1)*BN); this CTA
         // supplies the rank-th half of each
         const int qcol0 = c.qb * TILE_N + static_cast<int>(rank) * HALF_N;
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_phase<true>(smem_u32(&empty_bar[s]), ph ^ 1u, ctl, p, kStatusTimeoutProducer)) {
@@ -238,13 +246,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       const uint32_t peer_empty0 = map_shared_rank(smem_u32(&empty_bar[0]), peer);
       const uint32_t peer_accf0 = map_shared_rank(smem_u32(&accf_bar[0]), peer);
-      for (long long t = pair_id; t < num_tiles && ok; t += num_pairs, ++local) {
+      WorkIter wi(p, num_tiles, sk_width, sk_tiles, pair_id, num_pairs);
+      Work w;
+      for (; ok && wi.next(p, w); ++local) {
         const uint32_t a = ACC_BUFS == 2 ? (local & 1u) : 0u;
         const uint32_t aph = ACC_BUFS == 2 ? ((local >> 1) & 1u) : (local & 1u);
         if (!wait_phase<true>(smem_u32(&acce_bar[a]), aph ^ 1u, ctl, p, kStatusTimeoutMma)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + a * TILE_N;
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        for (int kb = w.kb0; kb < w.kb1; ++kb, ++it) {
           const uint32_t s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!wait_phase<true>(smem_u32(&full_bar[s]), ph, ctl, p, kStatusTimeoutMma)) {
@@ -263,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t qb_addr = qbase + sub * QSUB_BYTES;
               const uint64_t bdesc = Q_MN ? sw128_desc(qb_addr + k * 16 * 128, kBK * 128, 1024)
                                           : sw128_desc(qb_addr + k * 32, 16, 1024);
-              mma_f16<2>(d + sub * BN, adesc, bdesc, IDESC, (kb | k) != 0 ? 1u : 0u);
+              mma_f16<2>(d + sub * BN, adesc, bdesc, IDESC, (kb != w.kb0 || k != 0) ? 1u : 0u);
             }
           }
           // stage s is free in both CTAs once these MMAs have read it
@@ -288,32 +298,113 @@ __global__ void __launch_bounds__(kThreads, 1)
     const InT* bias = (p.epi & 1) ? reinterpret_cast<const InT*>(p.bias) : nullptr;
     const bool relu = (p.epi & 2) != 0;
     const uint32_t acce_leader0 = map_shared_rank(smem_u32(&acce_bar[0]), 0);
+    const int row_local = quad * 32 + lane;  // this thread's accumulator row in this CTA
+    const bool pieces_possible = p.work_mode != 0;  // uniform for the launch
+    constexpr long long PART = static_cast<long long>(kBM) * TILE_N;  // floats per CTA partial
+    // this warp is done reading accumulator `a`
+    auto free_acc = [&](uint32_t a) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(acce_leader0 + a * 8u);
+    };
     int gcur = 0;
-    for (long long t = pair_id; t < num_tiles; t += num_pairs, ++local) {
-      const PairTile c = pair_tile(t, gcur);
+    WorkIter wi(p, num_tiles, sk_width, sk_tiles, pair_id, num_pairs);
+    Work w;
+    for (; wi.next(p, w); ++local) {
+      const PairTile c = pair_tile(w.t, gcur);
       const long long b = c.b;
       const int qb = c.qb;
       const InT* const bias_t =
           bias ? bias + b * (GROUPED ? static_cast<long long>(p.N) : p.stride_bias) : nullptr;
       const uint32_t a = ACC_BUFS == 2 ? (local & 1u) : 0u;
       const uint32_t aph = ACC_BUFS == 2 ? ((local >> 1) & 1u) : (local & 1u);
+      BiasRegs<TILE_N, InT> br;
+      if (!GROUPED) br.load(bias_t, qb * TILE_N, p.N);
       const bool ok = wait_phase<true>(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      if (pieces_possible) {
+        // the piece path syncs the four epilogue warps: one answer for all
+        if (epilogue_bar_any(!ok || *reinterpret_cast<volatile int*>(&ctl->abort))) break;
+      } else if (!__all_sync(0xffffffffu, ok)) {
+        break;
+      }
       if (warp == 2 && lane == 0 && local == 0) trace_mark(p, kTrFirstEpi);
       tc_fence_after();
       const int row0 = c.p0 + static_cast<int>(rank) * kBM + quad * 32;
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + a * TILE_N;
       const TmemSrc tsrc{taddr};
-      if (!GROUPED && p.tma_store)
-        store_tma_from<TILE_N, InT, OutT>(tsrc, row0, qb * TILE_N, static_cast<int>(b), p, bias_t,
-                                          relu, stage, stores, &tmC);
-      else
+      const long long cidx = 2 * w.t + rank;  // this CTA's counter for the tile
+      const long long first_pair = pair_id - w.idx;
+      bool finish = true;
+      if (w.count > 1) {
+        // one piece of a split tile: arrive on the counter (low 16 bits);
+        // the last to arrive sums, every other piece parks its partial and
+        // counts it written (high 16 bits)
+        epilogue_bar();
+        if (row_local == 0) {
+          const unsigned old = atomicAdd(&p.counters[cidx], 1u);
+          ctl->last = ((old & 0xFFFFu) == static_cast<unsigned>(w.count - 1)) ? 1 : 0;
+        }
+        epilogue_bar();
+        finish = ctl->last != 0;
+        if (!finish) {
+          float* part = p.ws + piece_slot(p, w.t, w.idx, first_pair, static_cast<int>(rank), 2) * PART;
+#pragma unroll 1
+          for (int cc = 0; cc < TILE_N; cc += 16) {
+            uint32_t v[16];
+            tsrc.get<16>(cc, v);
+            put_partial16(part, row_local, cc, v);
+          }
+          free_acc(a);  // the accumulator is free again
+          __threadfence();
+          epilogue_bar();
+          if (row_local == 0) atomicAdd(&p.counters[cidx], 0x10000u);
+        } else {
+          bool gave_up = false;
+          if (row_local == 0) {
+            // every other piece has arrived and writes its partial without
+            // waiting on anything: a bounded wait
+            const unsigned need = static_cast<unsigned>(w.count - 1);
+            const volatile unsigned* cnt = p.counters + cidx;
+            const uint64_t t0 = global_timer_ns();
+            while ((*cnt >> 16) < need) {
+              if (global_timer_ns() - t0 > p.timeout_ns) {
+                atomicCAS(p.status, 0u, kStatusTimeoutEpilogue);
+                *reinterpret_cast<volatile int*>(&ctl->abort) = 1;
+                gave_up = true;
+                break;
+              }
+            }
+            __threadfence();
+          }
+          if (epilogue_bar_any(gave_up)) break;
+        }
+      }
+      if (!finish) continue;
+      if (w.count > 1) {
+        const PieceSumSrc psrc{tsrc, &p, w.t, first_pair, PART, w.count, w.idx, row_local,
+                               static_cast<int>(rank), 2};
+        if (!GROUPED && p.tma_store)
+          store_tma_from<TILE_N, InT, OutT>(psrc, row0, qb * TILE_N, static_cast<int>(b), p, bias_t,
+                                            relu, stage, stores, &tmC);
+        else
+          store_rows_from<TILE_N, InT, OutT>(
+              psrc, row0 + lane, c.row_end, qb * TILE_N, p, bias_t, relu,
+              reinterpret_cast<OutT*>(p.C) + (GROUPED ? 0 : b * p.stride_c));
+        if (row_local == 0) p.counters[cidx] = 0u;  // ready for the next launch
+      } else if (!GROUPED && p.tma_store) {
+        if (bias_t != nullptr)
+          store_tmem_tile<TILE_N, InT, OutT, true>(taddr, row0, qb * TILE_N, static_cast<int>(b),
+                                                   p, br, relu, stage, stores, &tmC);
+        else
+          store_tmem_tile<TILE_N, InT, OutT, false>(taddr, row0, qb * TILE_N,
+                                                    static_cast<int>(b), p, br, relu, stage,
+                                                    stores, &tmC);
+      } else {
         store_rows_from<TILE_N, InT, OutT>(
             tsrc, row0 + lane, c.row_end, qb * TILE_N, p, bias_t, relu,
             reinterpret_cast<OutT*>(p.C) + (GROUPED ? 0 : b * p.stride_c));
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(acce_leader0 + a * 8u);
+      }
+      free_acc(a);
     }
     if (!GROUPED && lane == 0) tma_store_wait_read<0>();  // staging read; writes finish with the grid
     if (warp == 2 && lane == 0) trace_mark(p, kTrEpiDone);

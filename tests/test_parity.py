@@ -79,7 +79,7 @@ def test_moe_grouped_sampled(config):
 @pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
 @pytest.mark.parametrize("b_col", [False, True])
 @pytest.mark.parametrize("config", [0, 1, 4, 5, 8, 9, 10, 11, 12, 13, 23, 24, 28, 29, 30, 31,
-                                    32, 34, 35])
+                                    32, 34, 35, 36, 37, 38])
 def test_exact_integers(dtype, b_col, config):
     """Integer inputs in [-2, 2] with K <= 4096: every partial sum is an
     exact integer below 2^24, so the fp32 accumulator is exact in any order
@@ -150,7 +150,7 @@ def test_empty_m_or_n_is_a_noop():
     assert bool((g.ibuf.cpu() == g.sent).all())
 
 
-DENSE_CONFIGS = list(range(25)) + list(range(28, 36))  # 25..27 are grouped-only
+DENSE_CONFIGS = list(range(25)) + list(range(28, 39))  # 25..27 are grouped-only
 
 
 @pytest.mark.parametrize("config", DENSE_CONFIGS)
@@ -177,6 +177,84 @@ def test_every_config_on_ragged_problem(config, dtype, out_f32):
         compare(g.matrix().double().cpu().numpy(), ref, 4 if out_f32 else 2,
                 f"{name} b_col={b_col}")
         g.check_canaries()
+
+
+PAIR_SK_CONFIGS = [36, 37, 38]  # CTA-pair stream-K, hybrid, and stream-K on 256 x 256 tiles
+
+
+@pytest.mark.parametrize("config", PAIR_SK_CONFIGS)
+@pytest.mark.parametrize("M,N,K,b_col", [(1000, 1504, 2000, False), (2304, 2560, 1536, True),
+                                         (777, 1104, 4104, False)])
+def test_pair_stream_k_every_element(config, M, N, K, b_col):
+    """Stream-K over CTA pairs: pieces cross tile edges, each CTA of a pair
+    fixes up its own 128 rows; every element against the oracle, and a
+    second launch (counters left at zero) is bit-identical."""
+    name = dg.gemm_config_name(config)
+    gen = torch.Generator().manual_seed(5000 + config + M)
+    A = torch.randn(M, K, generator=gen).to(torch.bfloat16)
+    B = torch.randn(*((N, K) if b_col else (K, N)), generator=gen).to(torch.bfloat16)
+    bias = torch.randn(N, generator=gen).to(torch.bfloat16)
+    ref = oracle.gemm(M, N, K, A, K, B, K if b_col else N, b_colmajor=b_col, bias=bias,
+                      relu=True, dtype="bf16", threads=THREADS)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        outs = [run_gemm(A.cuda(), B.cuda(), bias.cuda(), M, N, K, b_col=b_col, relu=True)
+                for _ in range(2)]
+    finally:
+        dg.gemm_force_config(-1)
+    first = outs[0].matrix().cpu()
+    assert torch.equal(outs[1].matrix().cpu(), first)
+    compare(first.double().numpy(), ref, 2, f"{name} {M}x{N}x{K}")
+    for g in outs:
+        g.check_canaries()
+
+
+@pytest.mark.parametrize("config", PAIR_SK_CONFIGS)
+@pytest.mark.parametrize("name", ["square4096_bf16", "square8192_f16"])
+def test_pair_stream_k_sampled(config, name):
+    w = workloads.get(name)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        _dense_case(w, sampled=True)
+    finally:
+        dg.gemm_force_config(-1)
+
+
+@pytest.mark.parametrize("config", [None, 0, 1, 11, 13, 28])
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("offset", [0, 1, 3])
+def test_bias_at_element_alignment(config, dtype, offset):
+    """The bias needs only its element alignment: a vector that starts 1 or 3
+    elements past a 16-byte boundary, with N not a multiple of 16, must give
+    the same result as an aligned one (the epilogue loads the tile's bias
+    with vector loads only where they are aligned and inside N)."""
+    if dtype == torch.float32 and config not in (None, 0, 1):
+        pytest.skip("fp32 inputs run on the single-CTA 128 x 128 / 128 x 256 tf32 tiles only")
+    M, N, K = 300, 1000, 192
+    gen = torch.Generator().manual_seed(7000 + offset + (config or 0))
+    A = torch.randint(-2, 3, (M, K), generator=gen).to(dtype)
+    B = torch.randint(-2, 3, (K, N), generator=gen).to(dtype)
+    bias = torch.randint(-4, 5, (N,), generator=gen).to(dtype)
+    ref = oracle.gemm(M, N, K, A, K, B, N, bias=bias, relu=True, dtype=in_name(A),
+                      threads=THREADS) if dtype != torch.float32 else \
+        oracle.gemm_f32(M, N, K, A, K, B, N, bias=bias, relu=True, threads=THREADS)
+    dbias = torch.zeros(N + 8, dtype=dtype, device="cuda")
+    dbias[offset:offset + N] = bias.cuda()
+    if config is not None:
+        assert dg.gemm_force_config(config) == 0
+    try:
+        g = run_gemm(A.cuda(), B.cuda(), dbias[offset:offset + N], M, N, K, relu=True,
+                     out_f32=dtype != torch.float32 and offset == 1)
+    finally:
+        dg.gemm_force_config(-1)
+    # small integers: every partial sum is exact in fp32 in any order, so an
+    # fp32 output equals the oracle and a 16-bit one its round-to-nearest-even
+    out_f32 = dtype == torch.float32 or offset == 1
+    expect = ref if out_f32 else torch.from_numpy(ref).to(dtype).double().numpy()
+    got = g.matrix().double().cpu().numpy()
+    assert np.array_equal(got, expect), \
+        dg.gemm_config_name(config) if config is not None else "table"
+    g.check_canaries()
 
 
 def test_swap_config_rejects_row_major_b():
@@ -619,7 +697,7 @@ class BatchGuard:
         assert bool((raw[mask] == self.sent).all()), "write outside the batch outputs"
 
 
-@pytest.mark.parametrize("config", [None, 0, 1, 4, 13, 8, 23, 2])
+@pytest.mark.parametrize("config", [None, 0, 1, 4, 13, 8, 23, 2, 36, 37])
 @pytest.mark.parametrize("b_col", [False, True])
 @pytest.mark.parametrize("share", ["none", "a", "b"])
 def test_strided_batched(config, b_col, share):
