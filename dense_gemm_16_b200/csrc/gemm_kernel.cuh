@@ -338,11 +338,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!finish) {
           float* part =
               p.ws + piece_slot(p, w.t, w.idx, static_cast<long long>(blockIdx.x) - w.idx) * PART;
+          // up to 64 columns per tensor-memory round trip
+          constexpr int PW = BN < 64 ? BN : 64;
 #pragma unroll 1
-          for (int cc = 0; cc < BN; cc += 16) {
-            uint32_t v[16];
-            tsrc.get<16>(cc, v);
-            put_partial16(part, row_local, cc, v);
+          for (int cc = 0; cc < BN; cc += PW) {
+            uint32_t v[PW];
+            tsrc.get<PW>(cc, v);
+#pragma unroll
+            for (int h = 0; h < PW; h += 16)
+              put_partial16(part, row_local, cc + h, *reinterpret_cast<uint32_t(*)[16]>(&v[h]));
           }
           tc_fence_before();
           mbar_arrive(smem_u32(&acce_bar[a]));  // the accumulator is free again
@@ -376,14 +380,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         if constexpr (!SWAP) {
           const InT* bias_g = bias_t;
           if (TMA_EPI && p.tma_store) {
-            if (w.count > 1)
-              store_tma_from<BN, InT, OutT>(psrc, c.p0 + quad * 32, q0, c.group, p, bias_g, relu,
-                                            stage, stores, &tmC);
+            if (w.count > 1 && bias_g != nullptr)
+              store_tile_from<BN, InT, OutT, true>(psrc, c.p0 + quad * 32, q0, c.group, p, br,
+                                                   relu, stage, stores, &tmC);
+            else if (w.count > 1)
+              store_tile_from<BN, InT, OutT, false>(psrc, c.p0 + quad * 32, q0, c.group, p, br,
+                                                    relu, stage, stores, &tmC);
             else if (bias_g != nullptr)
-              store_tmem_tile<BN, InT, OutT, true>(taddr, c.p0 + quad * 32, q0, c.group, p, br,
+              store_tile_from<BN, InT, OutT, true>(tsrc, c.p0 + quad * 32, q0, c.group, p, br,
                                                    relu, stage, stores, &tmC);
             else
-              store_tmem_tile<BN, InT, OutT, false>(taddr, c.p0 + quad * 32, q0, c.group, p, br,
+              store_tile_from<BN, InT, OutT, false>(tsrc, c.p0 + quad * 32, q0, c.group, p, br,
                                                     relu, stage, stores, &tmC);
           } else {
             // accumulator row = output row prow, columns q0 .. q0+BN

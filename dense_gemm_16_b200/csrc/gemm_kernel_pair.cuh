@@ -348,11 +348,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         finish = ctl->last != 0;
         if (!finish) {
           float* part = p.ws + piece_slot(p, w.t, w.idx, first_pair, static_cast<int>(rank), 2) * PART;
+          // up to 64 columns per tensor-memory round trip
+          constexpr int PW = TILE_N < 64 ? TILE_N : 64;
 #pragma unroll 1
-          for (int cc = 0; cc < TILE_N; cc += 16) {
-            uint32_t v[16];
-            tsrc.get<16>(cc, v);
-            put_partial16(part, row_local, cc, v);
+          for (int cc = 0; cc < TILE_N; cc += PW) {
+            uint32_t v[PW];
+            tsrc.get<PW>(cc, v);
+#pragma unroll
+            for (int h = 0; h < PW; h += 16)
+              put_partial16(part, row_local, cc + h, *reinterpret_cast<uint32_t(*)[16]>(&v[h]));
           }
           free_acc(a);  // the accumulator is free again
           __threadfence();
@@ -383,20 +387,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (w.count > 1) {
         const PieceSumSrc psrc{tsrc, &p, w.t, first_pair, PART, w.count, w.idx, row_local,
                                static_cast<int>(rank), 2};
-        if (!GROUPED && p.tma_store)
-          store_tma_from<TILE_N, InT, OutT>(psrc, row0, qb * TILE_N, static_cast<int>(b), p, bias_t,
-                                            relu, stage, stores, &tmC);
-        else
+        if (!GROUPED && p.tma_store) {
+          if (bias_t != nullptr)
+            store_tile_from<TILE_N, InT, OutT, true>(psrc, row0, qb * TILE_N, static_cast<int>(b),
+                                                     p, br, relu, stage, stores, &tmC);
+          else
+            store_tile_from<TILE_N, InT, OutT, false>(psrc, row0, qb * TILE_N,
+                                                      static_cast<int>(b), p, br, relu, stage,
+                                                      stores, &tmC);
+        } else
           store_rows_from<TILE_N, InT, OutT>(
               psrc, row0 + lane, c.row_end, qb * TILE_N, p, bias_t, relu,
               reinterpret_cast<OutT*>(p.C) + (GROUPED ? 0 : b * p.stride_c));
         if (row_local == 0) p.counters[cidx] = 0u;  // ready for the next launch
       } else if (!GROUPED && p.tma_store) {
         if (bias_t != nullptr)
-          store_tmem_tile<TILE_N, InT, OutT, true>(taddr, row0, qb * TILE_N, static_cast<int>(b),
+          store_tile_from<TILE_N, InT, OutT, true>(tsrc, row0, qb * TILE_N, static_cast<int>(b),
                                                    p, br, relu, stage, stores, &tmC);
         else
-          store_tmem_tile<TILE_N, InT, OutT, false>(taddr, row0, qb * TILE_N,
+          store_tile_from<TILE_N, InT, OutT, false>(tsrc, row0, qb * TILE_N,
                                                     static_cast<int>(b), p, br, relu, stage,
                                                     stores, &tmC);
       } else {

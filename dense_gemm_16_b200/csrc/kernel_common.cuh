@@ -585,14 +585,13 @@ struct BiasRegs {
   }
 };
 
-// store_tma_from for a tensor-memory accumulator: the same chunks, with the
-// chunk loop unrolled and the bias taken from registers loaded ahead of time
-// (BIAS: add `br`), so each chunk's TMEM load, rounding, staging and TMA
-// store are straight-line code with no global load on the way.  Measured on
-// the 256 x 512 pair tile, whose MMA waits for this store: 5 us per tile
-// against 8.8 us for the generic loop.
-template <int TILE_N, typename InT, typename OutT, bool BIAS>
-__device__ __forceinline__ void store_tmem_tile(uint32_t taddr, int row0, int q0, int z,
+// store_tma_from with the chunk loop unrolled and the bias taken from
+// registers loaded ahead of time (BIAS: add `br`), so each chunk's source
+// read, rounding, staging and TMA store are straight-line code with no
+// global load on the way.  Measured on the 256 x 512 pair tile, whose MMA
+// waits for this store: 5 us per tile against 8.8 us for the generic loop.
+template <int TILE_N, typename InT, typename OutT, bool BIAS, typename Src>
+__device__ __forceinline__ void store_tile_from(const Src& src, int row0, int q0, int z,
                                                 const KParams& p, const BiasRegs<TILE_N, InT>& br,
                                                 bool relu, uint32_t stage, uint32_t& count,
                                                 const CUtensorMap* tmC) {
@@ -608,11 +607,7 @@ __device__ __forceinline__ void store_tmem_tile(uint32_t taddr, int row0, int q0
     if (c >= nch) break;  // warp-uniform
     const int col0 = q0 + c * CH;
     uint32_t v[CH];
-#pragma unroll
-    for (int h = 0; h < CH; h += 32)
-      tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(c * CH + h),
-                         *reinterpret_cast<uint32_t(*)[32]>(&v[h]));
-    tmem_ld_wait();
+    src.template get<CH>(c * CH, v);
     uint32_t packed[32];
     if constexpr (sizeof(OutT) == 2) {
 #pragma unroll

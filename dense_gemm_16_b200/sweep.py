@@ -140,6 +140,8 @@ def _grouped_calls(dg, torch, names, E, R, N, K, dtype):
     for cid, name in enumerate(names):
         if name.startswith(("swap", "csk", "pair_256x128")) or "_k" in name:
             skipped[cid] = "not a grouped kernel (or split-K, which grouped ignores)"
+        elif name.startswith("pair") and name.endswith(("_sk", "_hy")):
+            skipped[cid] = "grouped CTA pairs run whole tiles (the same kernel as without _sk/_hy)"
         else:
             calls[cid] = call
     return calls, skipped, keep
@@ -169,11 +171,13 @@ def run(reps=10, rounds=5, log=None, only=None, sustained=False):
         times, errors = _bench_rounds(dg, torch, calls, reps, rounds, flush)
         errors.update(skipped)
         row = {"class": cname, "M": M, "N": N, "K": K, "dtype": dtype, "b_col": b_col,
-               "grouped": grouped, "times_ms": {names[c]: t for c, t in times.items()},
+               "grouped": grouped, "sustained": sustained,
+               "times_ms": {names[c]: t for c, t in times.items()},
                "errors": {names[c]: e for c, e in errors.items()}}
         best = min(times, key=times.get)
         row["best"] = names[best]
         row["best_id"] = best
+        row["ids"] = {names[c]: c for c in times}
         row["best_tflops"] = 2.0 * M * N * K / (times[best] * 1e-3) / 1e12
         results.append(row)
         print(json.dumps(row), flush=True)
@@ -185,24 +189,47 @@ def run(reps=10, rounds=5, log=None, only=None, sustained=False):
     return results
 
 
+# A new winner replaces the incumbent of a class only if it is faster by more
+# than this fraction in the same sweep (run-to-run noise is about 1%).
+KEEP_MARGIN = 0.01
+
+
+def _rule_line(r, cid, name):
+    t = r["times_ms"][name]
+    tflops = 2.0 * r["M"] * r["N"] * r["K"] / (t * 1e-3) / 1e12
+    tag = " (sustained)" if r.get("sustained") else ""
+    return (f"    {{{r['M']}, {r['M']}, {r['N']}, {r['N']}, {r['K']}, {r['K']}, "
+            f"{int(r['b_col'])}, {int(r.get('grouped', False))}, {cid}}},  "
+            f"// {r['class']}{tag}: {name} {tflops:.0f} TFLOP/s")
+
+
 def write_rules(results, path=TABLE):
     """Rewrite the RULES block: one exact-shape rule per swept class.  Rules
-    of classes not in `results` are kept as they are."""
+    of classes not in `results` are kept as they are; so is a class's rule
+    when its config is within KEEP_MARGIN of the sweep's best, and a rule
+    chosen under sustained load when the new sweep was not (a burst sweep
+    does not overrule it)."""
     text = open(path).read()
     m = re.search(r"// BEGIN RULES \(written by the sweep\)\n(.*?)// END RULES", text, flags=re.S)
-    old = {}
+    old = {}  # class -> (line, config name, sustained)
     for line in m.group(1).splitlines():
-        c = re.search(r"//\s*([^:]+):", line)
+        c = re.search(r"//\s*([^:(]+?)\s*(\(sustained\))?:\s*(\S+)", line)
         if c and line.strip().startswith("{"):
-            old[c.group(1)] = line
+            old[c.group(1)] = (line, c.group(3), c.group(2) is not None)
     new = {}
     for r in results:
-        new[r["class"]] = (
-            f"    {{{r['M']}, {r['M']}, {r['N']}, {r['N']}, {r['K']}, {r['K']}, "
-            f"{int(r['b_col'])}, {int(r.get('grouped', False))}, {r['best_id']}}},  "
-            f"// {r['class']}: {r['best']} "
-            f"{r['best_tflops']:.0f} TFLOP/s")
-    merged = dict(old)
+        best_name, best_id = r["best"], r["best_id"]
+        inc = old.get(r["class"])
+        if inc is not None:
+            _, inc_name, inc_sustained = inc
+            if inc_sustained and not r.get("sustained"):
+                continue  # keep the rule measured under sustained load
+            if inc_name in r["times_ms"] and \
+                    r["times_ms"][best_name] >= (1.0 - KEEP_MARGIN) * r["times_ms"][inc_name]:
+                best_name = inc_name
+                best_id = _config_id(inc_name, r, best_id)
+        new[r["class"]] = _rule_line(r, best_id, best_name)
+    merged = {k: v[0] for k, v in old.items()}
     merged.update(new)
     lines = ["static const Rule kRules[] = {"] + list(merged.values())
     lines.append("    {0, 0, 0, 0, 0, 0, -1, -1, -1},  // sentinel")
@@ -211,6 +238,16 @@ def write_rules(results, path=TABLE):
                  lambda mm: mm.group(1) + "\n".join(lines) + "\n" + mm.group(2), text, flags=re.S)
     with open(path, "w") as f:
         f.write(out)
+
+
+def _config_id(name, row, fallback):
+    """The config id of `name`: from the row's id map when the sweep recorded
+    one, else from the compiled table's names in config_table.h."""
+    ids = row.get("ids")
+    if ids and name in ids:
+        return ids[name]
+    names = re.findall(r'^\s*\{"([^"]+)",', open(TABLE).read(), flags=re.M)
+    return names.index(name) if name in names else fallback
 
 
 def main(argv=None):

@@ -225,3 +225,61 @@ def test_trace_setting_checks_alignment_and_turns_off():
     assert dg.gemm_set_trace(None, 0) == dg.GEMM_OK
     assert dg.gemm_set_trace(0x1000, 8) == dg.GEMM_OK  # too small for one block: off
     assert dg.GEMM_TRACE_EVENTS == 8 and dg.GEMM_TRACE_EXIT == 7
+
+
+# ------------------------------------------------ the sweep's rule writer
+
+_TABLE = """// head
+// BEGIN RULES (written by the sweep)
+static const Rule kRules[] = {
+    {64, 64, 64, 64, 64, 64, 0, 0, 1},  // sq64: cfgB 10 TFLOP/s
+    {96, 96, 96, 96, 96, 96, 0, 0, 1},  // sq96 (sustained): cfgB 20 TFLOP/s
+    {0, 0, 0, 0, 0, 0, -1, -1, -1},  // sentinel
+};
+// END RULES
+// tail
+"""
+
+
+def _row(cls, n, times, sustained=False):
+    best = min(times, key=times.get)
+    ids = {"cfgA": 0, "cfgB": 1, "cfgC": 2}
+    return {"class": cls, "M": n, "N": n, "K": n, "b_col": False, "grouped": False,
+            "sustained": sustained, "times_ms": times, "best": best, "best_id": ids[best],
+            "best_tflops": 0.0, "ids": ids}
+
+
+def _rules(path):
+    import re
+    text = open(path).read()
+    found = re.findall(r"^\s*\{(\d+), .*?, (-?\d+)\},  // ([^\n]+)$", text, flags=re.M)
+    return [f for f in found if f[2] != "sentinel"], text
+
+
+def test_sweep_rule_writer(tmp_path):
+    from dense_gemm_16_b200 import sweep
+    path = tmp_path / "table.h"
+    path.write_text(_TABLE)
+    sweep.write_rules([
+        _row("sq64", 64, {"cfgA": 0.995, "cfgB": 1.0}),     # within the margin: keep cfgB
+        _row("sq96", 96, {"cfgA": 0.5, "cfgB": 1.0}),       # burst sweep: keep the sustained rule
+        _row("sq128", 128, {"cfgC": 0.5, "cfgB": 1.0}),     # new class
+    ], path=str(path))
+    rules, text = _rules(path)
+    by_m = {int(m): (int(cid), note) for m, cid, note in rules}
+    assert by_m[64][0] == 1 and "sq64: cfgB" in by_m[64][1]
+    assert by_m[96] == (1, "sq96 (sustained): cfgB 20 TFLOP/s")
+    assert by_m[128][0] == 2 and "sq128: cfgC" in by_m[128][1]
+    assert text.startswith("// head") and text.rstrip().endswith("// tail")
+    assert "sentinel" in text and len(rules) == 3
+    # a clear win replaces the incumbent; a sustained sweep replaces a
+    # sustained rule, once, with the tag kept
+    sweep.write_rules([
+        _row("sq64", 64, {"cfgA": 0.9, "cfgB": 1.0}),
+        _row("sq96", 96, {"cfgC": 0.5, "cfgB": 1.0}, sustained=True),
+    ], path=str(path))
+    rules, _ = _rules(path)
+    by_m = {int(m): (int(cid), note) for m, cid, note in rules}
+    assert by_m[64][0] == 0 and "sq64: cfgA" in by_m[64][1]
+    assert by_m[96][0] == 2 and by_m[96][1].startswith("sq96 (sustained): cfgC")
+    assert len(rules) == 3
