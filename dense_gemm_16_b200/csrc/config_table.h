@@ -77,9 +77,9 @@ static const Rule kRules[] = {
     {1000, 1000, 1000, 1000, 2000, 2000, 1, 0, 31},  // m1000n1000k2000_bcol: csk_2x128x128_s4 217 TFLOP/s
     {4096, 4096, 4096, 4096, 512, 512, 1, 0, 0},  // m4096n4096k512_bcol: tc1_128x256_s4_g8 684 TFLOP/s
     {16, 16, 8192, 8192, 8192, 8192, 1, 0, 21},  // m16n8192k8192_bcol: swap_128x16_s8_sk 62 TFLOP/s
-    {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 699 TFLOP/s
-    {16384, 16384, 4096, 4096, 4096, 4096, 0, 1, 4},  // moe8_n4096_k4096: pair_256x256_s6_g8 1240 TFLOP/s
-    {8192, 8192, 768, 768, 2048, 2048, 0, 1, 11},  // moe64_n768_k2048: pair_256x256_s6_g16 393 TFLOP/s
+    {8192, 8192, 1408, 1408, 4096, 4096, 0, 1, 0},  // moe32_n1408_k4096: tc1_128x256_s4_g8 669 TFLOP/s
+    {16384, 16384, 4096, 4096, 4096, 4096, 0, 1, 12},  // moe8_n4096_k4096: pair_256x512_s4_g8 1288 TFLOP/s
+    {8192, 8192, 768, 768, 2048, 2048, 0, 1, 11},  // moe64_n768_k2048: pair_256x256_s6_g16 405 TFLOP/s
     {0, 0, 0, 0, 0, 0, -1, -1, -1},  // sentinel
 };
 // END RULES

@@ -942,7 +942,10 @@ int grouped_gemm(int num_groups, const int32_t* group_rows, int total_rows, int 
   CUtensorMap tc;
   std::memset(&tc, 0, sizeof(tc));  // grouped tiles store from registers
   if (pair) {
-    // 256-row pair tiles; one cluster of two CTAs per pair
+    // 256-row pair tiles; one cluster of two CTAs per pair.  Rows whose N
+    // columns are whole 16-byte vectors leave by vector stores of staged
+    // row segments (flag reused from the dense TMA store)
+    kp.tma_store = (static_cast<int64_t>(N) * (f32 ? 4 : 2)) % 16 == 0 ? 1 : 0;
     const long long max_pair_tiles =
         (static_cast<long long>(total_rows) / (2 * kBM) + num_groups) * nq;
     const int pairs = static_cast<int>(std::min<long long>(max_pair_tiles, ds->num_sms / 2));

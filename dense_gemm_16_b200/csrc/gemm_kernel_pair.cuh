@@ -52,9 +52,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t Q_BYTES = NSUB * QSUB_BYTES;
   constexpr uint32_t STAGE_BYTES = P_BYTES + Q_BYTES;
   constexpr uint32_t TMEM_COLS = (ACC_BUFS * TILE_N <= 256) ? 256 : 512;
-  // grouped tiles must not write past their group's last row: they store
-  // from registers and need no staging buffer
-  constexpr uint32_t STAGE_EPI = GROUPED ? 0u : kEpiStageBytes;
+  // grouped tiles must not write past their group's last row: they stage
+  // through one 4 KB buffer per epilogue warp and store masked rows
+  constexpr uint32_t STAGE_EPI = GROUPED ? kEpiStageBytes / 2 : kEpiStageBytes;
   constexpr uint32_t IDESC = f16_idesc(2 * kBM, BN, IN_BF16 ? 1u : 0u, 0u, Q_MN ? 1u : 0u);
 
   extern __shared__ uint8_t smem_raw[];
@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // --------------------------------------------- epilogue (both CTAs)
     const int quad = warp & 3;
-    const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>(warp - 2) * 8192u;
+    const uint32_t stage = smem_u32(sStage) + static_cast<uint32_t>(warp - 2) * (STAGE_EPI / 4);
     uint32_t stores = 0;
     uint32_t local = 0;
     const InT* bias = (p.epi & 1) ? reinterpret_cast<const InT*>(p.bias) : nullptr;
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t a = ACC_BUFS == 2 ? (local & 1u) : 0u;
       const uint32_t aph = ACC_BUFS == 2 ? ((local >> 1) & 1u) : (local & 1u);
       BiasRegs<TILE_N, InT> br;
-      if (!GROUPED) br.load(bias_t, qb * TILE_N, p.N);
+      br.load(bias_t, qb * TILE_N, p.N);
       const bool ok = wait_phase<true>(smem_u32(&accf_bar[a]), aph, ctl, p, kStatusTimeoutEpilogue);
       if (pieces_possible) {
         // the piece path syncs the four epilogue warps: one answer for all
@@ -408,6 +408,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           store_tile_from<TILE_N, InT, OutT, false>(tsrc, row0, qb * TILE_N,
                                                     static_cast<int>(b), p, br, relu, stage,
                                                     stores, &tmC);
+      } else if (GROUPED && p.tma_store) {
+        // grouped: masked at the group's last row (tma_store: N whole 16-byte vectors)
+        OutT* const Cg = reinterpret_cast<OutT*>(p.C);
+        if (bias_t != nullptr)
+          store_tile_rows<TILE_N, InT, OutT, true>(tsrc, row0, c.row_end, qb * TILE_N, p, br, relu,
+                                                   stage, Cg);
+        else
+          store_tile_rows<TILE_N, InT, OutT, false>(tsrc, row0, c.row_end, qb * TILE_N, p, br,
+                                                    relu, stage, Cg);
       } else {
         store_rows_from<TILE_N, InT, OutT>(
             tsrc, row0 + lane, c.row_end, qb * TILE_N, p, bias_t, relu,
@@ -433,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int BN, int NSUB, int STAGES, bool GROUPED = false>
 constexpr int gemm_pair_smem_bytes() {
   return 1024 + STAGES * (kBM * kBK * 2 + NSUB * (BN / 2) * kBK * 2) +
-         (GROUPED ? 0 : static_cast<int>(kEpiStageBytes)) + (2 * STAGES + 5) * 8 +
+         static_cast<int>(GROUPED ? kEpiStageBytes / 2 : kEpiStageBytes) + (2 * STAGES + 5) * 8 +
          static_cast<int>(sizeof(SharedCtl)) + (GROUPED ? static_cast<int>(sizeof(GroupTable)) : 0);
 }
 

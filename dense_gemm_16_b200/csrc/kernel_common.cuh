@@ -667,6 +667,90 @@ __device__ __forceinline__ void store_tile_from(const Src& src, int row0, int q0
   }
 }
 
+// store_tile_from for tiles whose rows may end inside the warp's 32 (a
+// grouped GEMM's last tile of a group): the same unrolled chunks, staged in
+// one 4 KB swizzled buffer per warp, then read back row-contiguously so each
+// vector store writes 16 bytes of a whole 128-byte row segment; rows at or
+// past row_end and columns at or past N are masked.  No TMA and nothing to
+// wait for.  Needs C 16-byte aligned and ldc and N multiples of 16 bytes.
+template <int TILE_N, typename InT, typename OutT, bool BIAS, typename Src>
+__device__ __forceinline__ void store_tile_rows(const Src& src, int row0, int row_end, int q0,
+                                                const KParams& p, const BiasRegs<TILE_N, InT>& br,
+                                                bool relu, uint32_t buf, OutT* C) {
+  constexpr int CH = 128 / static_cast<int>(sizeof(OutT));  // outputs per 128-byte row chunk
+  constexpr int NCH = TILE_N / CH;
+  constexpr int EPV = 16 / static_cast<int>(sizeof(OutT));  // outputs per 16-byte vector
+  static_assert(TILE_N % CH == 0, "whole chunks");
+  const int lane = threadIdx.x & 31;
+  const int nch = row0 >= row_end ? 0 : max(0, min(NCH, (p.N - q0 + CH - 1) / CH));
+  const int sl = lane & 7;  // read-back: this lane's 16-byte slot of a row
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    if (c >= nch) break;  // warp-uniform
+    uint32_t v[CH];
+    src.template get<CH>(c * CH, v);
+    uint32_t packed[32];
+    if constexpr (sizeof(OutT) == 2) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        float x0 = __uint_as_float(v[2 * j]), x1 = __uint_as_float(v[2 * j + 1]);
+        if constexpr (BIAS) {
+          float b0, b1;
+          br.pair(c * CH + 2 * j, b0, b1);
+          x0 += b0;
+          x1 += b1;
+        }
+        if (relu) {
+          x0 = fmaxf(x0, 0.0f);
+          x1 = fmaxf(x1, 0.0f);
+        }
+        packed[j] = pack2<OutT>(x0, x1);
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; j += 2) {
+        float x0 = __uint_as_float(v[j]), x1 = __uint_as_float(v[j + 1]);
+        if constexpr (BIAS) {
+          float b0, b1;
+          br.pair(c * CH + j, b0, b1);
+          x0 += b0;
+          x1 += b1;
+        }
+        if (relu) {
+          x0 = fmaxf(x0, 0.0f);
+          x1 = fmaxf(x1, 0.0f);
+        }
+        packed[j] = __float_as_uint(x0);
+        packed[j + 1] = __float_as_uint(x1);
+      }
+    }
+    __syncwarp();  // the previous chunk's read-back of the buffer is done
+    const uint32_t row_addr = buf + static_cast<uint32_t>(lane) * 128u;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const uint32_t dst = row_addr + ((static_cast<uint32_t>(q) ^ (lane & 7u)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(packed[4 * q]),
+                   "r"(packed[4 * q + 1]), "r"(packed[4 * q + 2]), "r"(packed[4 * q + 3])
+                   : "memory");
+    }
+    __syncwarp();
+    const int col = q0 + c * CH + sl * EPV;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = 4 * i + (lane >> 3);  // rows 4i .. 4i+3, eight lanes each
+      uint32_t x0, x1, x2, x3;
+      asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                   : "=r"(x0), "=r"(x1), "=r"(x2), "=r"(x3)
+                   : "r"(buf + static_cast<uint32_t>(r) * 128u +
+                         ((static_cast<uint32_t>(sl) ^ static_cast<uint32_t>(r & 7)) << 4))
+                   : "memory");
+      if (row0 + r < row_end && col < p.N)
+        *reinterpret_cast<uint4*>(C + static_cast<long long>(row0 + r) * p.ldc + col) =
+            make_uint4(x0, x1, x2, x3);
+    }
+  }
+}
+
 // TMEM as a source of raw accumulator values for the epilogues above: the
 // warp's 32 lanes x 16 consecutive columns starting at `taddr + cc`.
 // get<W>(cc, v) fills v with W consecutive columns starting at cc; all

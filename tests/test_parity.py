@@ -500,6 +500,42 @@ def test_grouped_every_element(b_col, out_f32, config):
     g.check_canaries()
 
 
+@pytest.mark.parametrize("config", [4, 11, 13])
+@pytest.mark.parametrize("N", [196, 200, 512, 1000])
+@pytest.mark.parametrize("out_f32", [False, True])
+def test_grouped_pair_stores_every_element(config, N, out_f32):
+    """Grouped CTA-pair tiles leave by staged row-segment stores masked at
+    each group's last row (N whole 16-byte vectors) or by per-row register
+    stores (N=196 in 16-bit); groups end inside a warp's 32 rows, inside a
+    CTA's 128 and inside a pair's 256."""
+    rows_per = np.array([0, 300, 256, 1, 511, 33], dtype=np.int32)
+    G, K = len(rows_per), 200
+    total = int(rows_per.sum())
+    gen = torch.Generator().manual_seed(90 + config + N)
+    X = torch.randn(total, K, generator=gen).bfloat16()
+    W = (torch.randn(G, N, K, generator=gen) * 0.1).bfloat16()  # column-major B: any N
+    bias = torch.randn(G, N, generator=gen).bfloat16()
+    ref = oracle.grouped_gemm(rows_per, N, K, X, K, W, K, N * K, b_colmajor=True, bias=bias,
+                              relu=True, dtype="bf16", threads=THREADS)
+    dt = torch.float32 if out_f32 else torch.bfloat16
+    ldc = (N + 15) // 8 * 8
+    g = Guarded(total, N, ldc, dt)
+    assert dg.gemm_force_config(config) == 0
+    try:
+        rc = dg.grouped_gemm(G, torch.from_numpy(rows_per).cuda(), total, N, K, X.cuda(), K,
+                             W.cuda(), K, N * K, g.ptr, ldc, bias.cuda(),
+                             dg.GEMM_EPI_BIAS | dg.GEMM_EPI_RELU | dg.GEMM_B_COL_MAJOR,
+                             dg.GEMM_BF16_OUT_F32 if out_f32 else dg.GEMM_BF16)
+    finally:
+        dg.gemm_force_config(-1)
+    assert rc == 0, dg.gemm_status_string(rc)
+    torch.cuda.synchronize()
+    assert dg.gemm_device_status() == 0
+    compare(g.matrix().double().cpu().numpy(), ref, 4 if out_f32 else 2,
+            f"{dg.gemm_config_name(config)} N={N}")
+    g.check_canaries()
+
+
 @pytest.mark.parametrize("config", [-1, 4, 13, 24, 25, 26])
 def test_grouped_counts_beyond_total_are_clipped_and_reported(config):
     rows_per = np.array([5, 300, 40], dtype=np.int32)  # sums to 345
