@@ -45,6 +45,11 @@
  *           Calls are asynchronous: GEMM_OK means the work was enqueued;
  *           a device-side fault shows up at the caller's next synchronisation,
  *           and a watchdog time-out is reported by gemm_device_status().
+ * Graphs.   Calls may be captured into a CUDA graph (stream capture).  A
+ *           capture cannot allocate, so make one uncaptured call of the same
+ *           shape and config on the capture stream first: it sizes that
+ *           stream's scratch.  Kernels leave their split-K / stream-K tile
+ *           counters at zero, so a graph replays any number of times.
  * Errors.   Every function returns a gemm_status; nothing throws, aborts or
  *           exits.  Argument errors are detected before anything is launched.
  * Threads.  All entry points are thread-safe.  The only mutable global state

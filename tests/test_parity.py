@@ -459,6 +459,69 @@ def test_runs_on_a_side_stream():
     compare(out.double().cpu().numpy(), ref, 2, "side stream")
 
 
+@pytest.mark.parametrize("config", [None, 8, 23, 36])
+def test_calls_replay_in_a_cuda_graph(config):
+    """gemm() and grouped_gemm() captured into one CUDA graph (after an
+    uncaptured call on the capture stream has sized its scratch) replay
+    correctly on fresh inputs, again and again: split-K and stream-K
+    counters are left at zero by every launch."""
+    name = dg.gemm_config_name(config) if config is not None else "table"
+    M, N, K = 640, 768, 1024
+    rows_per = np.array([100, 0, 300, 240], dtype=np.int32)
+    G, total = len(rows_per), int(rows_per.sum())
+    dA = torch.empty(M, K, dtype=torch.bfloat16, device="cuda")
+    dB = torch.empty(K, N, dtype=torch.bfloat16, device="cuda")
+    dbias = torch.empty(N, dtype=torch.bfloat16, device="cuda")
+    dC = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    dX = torch.empty(total, K, dtype=torch.bfloat16, device="cuda")
+    dW = torch.empty(G, K, N, dtype=torch.bfloat16, device="cuda")
+    dY = torch.empty(total, N, dtype=torch.bfloat16, device="cuda")
+    drows = torch.from_numpy(rows_per).cuda()
+    epi = dg.GEMM_EPI_BIAS | dg.GEMM_EPI_RELU
+    s = torch.cuda.Stream()
+
+    def calls():
+        rc = dg.gemm(M, N, K, dA, K, dB, N, dC, N, dbias, epi, dg.GEMM_BF16, s)
+        assert rc == 0, dg.gemm_status_string(rc)
+        rc = dg.grouped_gemm(G, drows, total, N, K, dX, K, dW, N, K * N, dY, N, None,
+                             dg.GEMM_EPI_RELU, dg.GEMM_BF16, s)
+        assert rc == 0, dg.gemm_status_string(rc)
+
+    if config is not None:
+        assert dg.gemm_force_config(config) == 0
+    try:
+        dA.zero_(); dB.zero_(); dbias.zero_(); dX.zero_(); dW.zero_()
+        torch.cuda.synchronize()
+        with torch.cuda.stream(s):
+            calls()  # sizes this stream's scratch outside the capture
+        s.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            calls()
+    finally:
+        dg.gemm_force_config(-1)
+    for rep in range(3):
+        gen = torch.Generator().manual_seed(8000 + rep + (config or 0))
+        A = torch.randn(M, K, generator=gen).bfloat16()
+        B = torch.randn(K, N, generator=gen).bfloat16()
+        bias = torch.randn(N, generator=gen).bfloat16()
+        X = torch.randn(total, K, generator=gen).bfloat16()
+        W = (torch.randn(G, K, N, generator=gen) * 0.1).bfloat16()
+        dA.copy_(A); dB.copy_(B); dbias.copy_(bias); dX.copy_(X); dW.copy_(W)
+        dC.fill_(float("nan")); dY.fill_(float("nan"))
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert dg.gemm_device_status() == 0
+        ref = oracle.gemm(M, N, K, A, K, B, N, bias=bias, relu=True, dtype="bf16",
+                          threads=THREADS)
+        compare(dC.double().cpu().numpy(), ref, 2, f"{name} graph replay {rep}")
+        refg = oracle.grouped_gemm(rows_per, N, K, X, K, W, N, K * N, relu=True, dtype="bf16",
+                                   threads=THREADS)
+        compare(dY.double().cpu().numpy(), refg, 2, f"{name} grouped graph replay {rep}")
+    del graph
+
+
 # --------------------------------------------------------------- grouped
 
 # 128 x 256 / 128 x 128 row tiles; swapped operands (one CTA, then CTA pairs)
