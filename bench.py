@@ -91,6 +91,38 @@ def _traffic(workload: str):
     return entry.get("dram_bytes_per_launch")
 
 
+def _roofline(flops: float, alg_bytes: float, ms_per_step: float, total_ms: float,
+              back_to_back: bool, dtype: str, peaks=None) -> dict:
+    """The roofline object of one bench line (traffic is added by the caller).
+
+    The bound is the slower of FLOPs at the dense tensor peak and the
+    algorithmic bytes at the HBM copy bandwidth.  Back-to-back launches for
+    half a second or more run under the power cap, so their tensor peak is
+    the sustained cuBLAS figure; otherwise the burst figure."""
+    peaks, peak_src = peaks if peaks is not None else _peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = back_to_back and total_ms >= 500.0
+    peak = float(peaks.get("bf16_tflops_sustained", burst)) if sustained else burst
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    t_tensor = flops / (peak * 1e12)
+    t_hbm = alg_bytes / (hbm * 1e9)
+    if t_hbm > t_tensor:
+        gbs = alg_bytes / (ms_per_step * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
+                "frac": round(gbs / hbm, 4), "peak_source": f"{peak_src} HBM copy bandwidth"}
+    else:
+        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_source": f"{peak_src} bf16 dense "
+                + ("(sustained: back-to-back launches under the power cap)" if sustained
+                   else "(burst)")
+                + ("; fp16 has the same dense rate" if dtype == "f16" else ""),
+                "frac_of_burst": round(achieved / burst, 4)}
+    roof["bound_times_us"] = {"tensor": round(t_tensor * 1e6, 2), "hbm": round(t_hbm * 1e6, 2)}
+    return roof
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -368,34 +400,13 @@ def bench_ours(args, rank, local, world):
     e2e_ms = _max_over_ranks(e_start.elapsed_time(e_stop), world, dev)
     e2e_value = flops * e2e_steps * world / (e2e_ms * 1e-3) / 1e12
 
-    peaks, peak_src = _peaks()
-    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    # Back-to-back launches for half a second or more run under the power cap:
-    # the tensor peak to compare with is then the sustained cuBLAS figure.
-    sustained = flush is None and total_ms >= 500.0
-    peak = float(peaks.get("bf16_tflops_sustained", burst)) if sustained else burst
-    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    roof = _roofline(flops, in_bytes + out_bytes, ms_per_step, total_ms, flush is None,
+                     w.dtype)
     alg_bytes = in_bytes + out_bytes
-    # the roofline is the slower of the two bounds: FLOPs at the dense tensor
-    # peak, or the algorithmic bytes at the HBM copy bandwidth
-    t_tensor = flops / (peak * 1e12)
-    t_hbm = alg_bytes / (hbm * 1e9)
-    if t_hbm > t_tensor:
-        gbs = alg_bytes / (ms_per_step * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": hbm, "unit": "GB/s",
-                "frac": round(gbs / hbm, 4), "peak_source": f"{peak_src} HBM copy bandwidth"}
-    else:
-        roof = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_source": f"{peak_src} bf16 dense "
-                + ("(sustained: back-to-back launches under the power cap)" if sustained
-                   else "(burst)")
-                + ("; fp16 has the same dense rate" if w.dtype == "f16" else ""),
-                "frac_of_burst": round(achieved / burst, 4)}
+    achieved = flops / (ms_per_step * 1e-3) / 1e12
+    burst = float(_peaks()[0].get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     roof["traffic"] = _traffic(w.name)
     roof["algorithmic_bytes"] = alg_bytes
-    roof["bound_times_us"] = {"tensor": round(t_tensor * 1e6, 2), "hbm": round(t_hbm * 1e6, 2)}
     result = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
