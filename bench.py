@@ -91,6 +91,16 @@ def _traffic(workload: str):
     return entry.get("dram_bytes_per_launch")
 
 
+def _workload_config(w, world: int) -> dict:
+    """The workload part of a bench line's `config`, the same for both arms
+    (our arm adds its L2 regime and the config the table chose)."""
+    return {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "in_dtype": w.dtype,
+            "acc_dtype": "f32", "out_dtype": w.out_dtype,
+            "b_layout": "col-major" if w.b_colmajor else "row-major",
+            "epilogue": ("bias+" if w.bias else "") + ("relu" if w.relu else "none"),
+            "experts": w.experts or None, "parallelism": f"replicas x{world}"}
+
+
 def _roofline(flops: float, alg_bytes: float, ms_per_step: float, total_ms: float,
               back_to_back: bool, dtype: str, peaks=None) -> dict:
     """The roofline object of one bench line (traffic is added by the caller).
@@ -412,17 +422,12 @@ def bench_ours(args, rank, local, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "f16", "data": "synthetic",
-        "config": {
-            "workload": w.name, "M": w.M, "N": w.N, "K": w.K, "in_dtype": w.dtype,
-            "acc_dtype": "f32", "out_dtype": w.out_dtype, "b_layout":
-                "col-major" if w.b_colmajor else "row-major",
-            "epilogue": ("bias+" if w.bias else "") + ("relu" if w.relu else "none"),
-            "experts": w.experts or None, "parallelism": f"replicas x{world}",
-            "l2": "flushed between steps (256 MiB write)" if flush is not None
-                  else f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB)",
-            "config_id": lib.gemm_select_config(w.M, w.N, w.K, code, epi) if not w.grouped
-            else None,
-        },
+        "config": dict(
+            _workload_config(w, world),
+            l2="flushed between steps (256 MiB write)" if flush is not None
+            else f"inputs larger than L2 ({in_bytes / 2**20:.0f} MiB)",
+            config_id=lib.gemm_select_config(w.M, w.N, w.K, code, epi) if not w.grouped
+            else None),
         "pct_of_peak": round(100.0 * achieved / burst, 2),
         "roofline": roof,
         "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d_bytes,
@@ -481,7 +486,7 @@ def bench_reference(args, rank, world):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "M": w.M, "N": w.N, "K": w.K, "in_dtype": w.dtype},
+        "config": _workload_config(w, world),
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": used, "kind": "oracle",
                          "sample": sample},

@@ -79,3 +79,19 @@ def test_traffic_dropped_once_a_kernel_source_changes(tmp_path, monkeypatch):
     assert bench._traffic("w") == 12345
     (csrc / "kernel.cu").write_text("// kernel v2\n")
     assert bench._traffic("w") is None
+
+
+def test_reference_arm_line_matches_the_contract(capsys):
+    """`bench.py --impl reference` (the oracle timed on the host cores) prints
+    one JSON line with our arm's metric, unit and workload config."""
+    import workloads
+    bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3",
+                "--workload", "square256_f16"])
+    lines = [ln for ln in capsys.readouterr().out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
+    assert d["higher_is_better"] is True and d["value"] > 0
+    assert d["config"] == bench._workload_config(workloads.get("square256_f16"), 1)
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
