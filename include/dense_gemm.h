@@ -215,6 +215,11 @@ GEMM_API const char* gemm_version(void);
  * and the kernel returned early; its output is undefined) or
  * GEMM_ERR_INVALID_ARG (grouped row counts were inconsistent).  With clear
  * != 0 the word is reset to 0 afterwards.
+ * After a time-out, the pieces of a split tile that gave up may have left
+ * that tile's counter set in the stream's scratch: call
+ * gemm_free_scratch(stream, 0) before the next split-K / stream-K call on
+ * that stream (the next call then allocates zeroed counters).
+ * gemm_splitk_noalloc clears its counters on every call and needs nothing.
  */
 GEMM_API int gemm_device_status(void* stream, int clear);
 
